@@ -1,0 +1,161 @@
+"""fp64 CPU oracle for exact attention -- TEST INFRASTRUCTURE ONLY.
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and bench.py's CPU-baseline leg may
+import this package. It wraps ``attn_oracle.c`` (plain C, double precision),
+which evaluates the naive definition S = scale*Q K^T (masked), P = softmax(S),
+O = P V, LSE = ln sum exp(S), plus per-chunk split-KV partials and their
+max-and-sum merge. It shares no code with the CUDA library.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import numpy as np
+
+from . import build as _build
+
+_c_long = ctypes.c_long
+_dp = ctypes.POINTER(ctypes.c_double)
+_fp = ctypes.POINTER(ctypes.c_float)
+_u16p = ctypes.POINTER(ctypes.c_uint16)
+_i64p = ctypes.POINTER(ctypes.c_int64)
+
+
+def _ptr(a: np.ndarray, t):
+    assert a.flags["C_CONTIGUOUS"]
+    return a.ctypes.data_as(t)
+
+
+class Oracle:
+    """ctypes handle on one build of the oracle library (normal or a mutant)."""
+
+    def __init__(self, path: str | None = None):
+        path = path or _build.build()
+        self.path = path
+        lib = ctypes.CDLL(path)
+        lib.oracle_attn_head_f64.argtypes = [_dp, _dp, _dp, _c_long, _c_long, _c_long,
+                                             ctypes.c_int, ctypes.c_double, _dp, _dp, _dp]
+        lib.oracle_attn_fwd_bf16.argtypes = [_u16p, _u16p, _u16p, _c_long, _c_long, _c_long,
+                                             _c_long, _c_long, ctypes.c_int, ctypes.c_double,
+                                             _dp, _dp]
+        lib.oracle_attn_rows_bf16.argtypes = [_u16p, _u16p, _u16p, _c_long, _c_long, _c_long,
+                                              ctypes.c_int, ctypes.c_double, _i64p, _c_long,
+                                              _dp, _dp]
+        lib.oracle_decode_partials_bf16.argtypes = [_u16p, _u16p, _u16p, _c_long, _c_long,
+                                                    ctypes.c_double, _c_long, _dp, _dp]
+        lib.oracle_lse_merge_f64.argtypes = [_dp, _dp, _c_long, _c_long, _dp, _dp]
+        lib.oracle_lse_merge_f32in.argtypes = [_fp, _fp, _c_long, _c_long, _c_long, _dp, _dp]
+        lib.oracle_num_threads.restype = ctypes.c_int
+        lib.oracle_set_num_threads.argtypes = [ctypes.c_int]
+        self.lib = lib
+
+    # -- double-precision entry (one head) ---------------------------------
+    def attn_head_f64(self, q, k, v, causal: bool, scale: float, want_p: bool = False):
+        q = np.ascontiguousarray(q, dtype=np.float64)
+        k = np.ascontiguousarray(k, dtype=np.float64)
+        v = np.ascontiguousarray(v, dtype=np.float64)
+        Nq, d = q.shape
+        Nkv = k.shape[0]
+        assert k.shape == (Nkv, d) and v.shape == (Nkv, d)
+        o = np.zeros((Nq, d))
+        lse = np.zeros(Nq)
+        p = np.zeros((Nq, Nkv)) if want_p else None
+        rc = self.lib.oracle_attn_head_f64(_ptr(q, _dp), _ptr(k, _dp), _ptr(v, _dp), Nq, Nkv,
+                                           d, int(causal), float(scale), _ptr(o, _dp),
+                                           _ptr(lse, _dp), _ptr(p, _dp) if want_p else None)
+        if rc:
+            raise RuntimeError("oracle_attn_head_f64 failed")
+        return (o, lse, p) if want_p else (o, lse)
+
+    # -- bf16 entries ---------------------------------------------------------
+    def attn_fwd_bf16(self, q_bits, k_bits, v_bits, causal: bool, scale: float):
+        """q_bits [B,H,Nq,d], k_bits/v_bits [B,H,Nkv,d] uint16 -> (O f64, LSE f64)."""
+        B, H, Nq, d = q_bits.shape
+        Nkv = k_bits.shape[2]
+        q, k, v = (np.ascontiguousarray(x, dtype=np.uint16) for x in (q_bits, k_bits, v_bits))
+        o = np.zeros((B, H, Nq, d))
+        lse = np.zeros((B, H, Nq))
+        rc = self.lib.oracle_attn_fwd_bf16(_ptr(q, _u16p), _ptr(k, _u16p), _ptr(v, _u16p), B, H,
+                                           Nq, Nkv, d, int(causal), float(scale),
+                                           _ptr(o, _dp), _ptr(lse, _dp))
+        if rc:
+            raise RuntimeError("oracle_attn_fwd_bf16 failed")
+        return o, lse
+
+    def attn_rows_bf16(self, q_head, k_head, v_head, rows, causal: bool, scale: float):
+        """One head: q_head [Nq,d], k_head/v_head [Nkv,d] uint16; rows: query indices."""
+        Nq, d = q_head.shape
+        Nkv = k_head.shape[0]
+        q, k, v = (np.ascontiguousarray(x, dtype=np.uint16) for x in (q_head, k_head, v_head))
+        r = np.ascontiguousarray(rows, dtype=np.int64)
+        o = np.zeros((len(r), d))
+        lse = np.zeros(len(r))
+        rc = self.lib.oracle_attn_rows_bf16(_ptr(q, _u16p), _ptr(k, _u16p), _ptr(v, _u16p), Nq,
+                                            Nkv, d, int(causal), float(scale), _ptr(r, _i64p),
+                                            len(r), _ptr(o, _dp), _ptr(lse, _dp))
+        if rc:
+            raise RuntimeError("oracle_attn_rows_bf16 failed")
+        return o, lse
+
+    def decode_partials_bf16(self, q_row, k_head, v_head, scale: float, num_splits: int):
+        d = q_row.shape[-1]
+        Nkv = k_head.shape[0]
+        q, k, v = (np.ascontiguousarray(x, dtype=np.uint16) for x in (q_row, k_head, v_head))
+        o = np.zeros((num_splits, d))
+        lse = np.zeros(num_splits)
+        rc = self.lib.oracle_decode_partials_bf16(_ptr(q, _u16p), _ptr(k, _u16p), _ptr(v, _u16p),
+                                                  Nkv, d, float(scale), num_splits,
+                                                  _ptr(o, _dp), _ptr(lse, _dp))
+        if rc:
+            raise RuntimeError("oracle_decode_partials_bf16 failed")
+        return o, lse
+
+    def lse_merge_f64(self, o_part, lse_part):
+        o_part = np.ascontiguousarray(o_part, dtype=np.float64)
+        lse_part = np.ascontiguousarray(lse_part, dtype=np.float64)
+        S, d = o_part.shape
+        o = np.zeros(d)
+        lse = np.zeros(1)
+        rc = self.lib.oracle_lse_merge_f64(_ptr(o_part, _dp), _ptr(lse_part, _dp), S, d,
+                                           _ptr(o, _dp), _ptr(lse, _dp))
+        if rc:
+            raise RuntimeError("oracle_lse_merge_f64 failed")
+        return o, float(lse[0])
+
+    def lse_merge_f32in(self, o_part, lse_part):
+        """o_part [B,H,S,d] f32, lse_part [B,H,S] f32 -> (O [B,H,d] f64, LSE [B,H] f64)."""
+        o_part = np.ascontiguousarray(o_part, dtype=np.float32)
+        lse_part = np.ascontiguousarray(lse_part, dtype=np.float32)
+        B, H, S, d = o_part.shape
+        o = np.zeros((B, H, d))
+        lse = np.zeros((B, H))
+        rc = self.lib.oracle_lse_merge_f32in(_ptr(o_part, _fp), _ptr(lse_part, _fp), B * H, S, d,
+                                             _ptr(o, _dp), _ptr(lse, _dp))
+        if rc:
+            raise RuntimeError("oracle_lse_merge_f32in failed")
+        return o, lse
+
+    def num_threads(self) -> int:
+        return int(self.lib.oracle_num_threads())
+
+    def set_num_threads(self, n: int) -> None:
+        self.lib.oracle_set_num_threads(int(n))
+
+
+_default: Oracle | None = None
+
+
+def get() -> Oracle:
+    """The oracle built from the unmodified source (built on first use)."""
+    global _default
+    if _default is None:
+        _default = Oracle()
+    return _default
+
+
+def build_mutant(n: int, out_dir: str) -> Oracle:
+    """A copy of the oracle with planted mistake ``n`` (1..9), for the pin tests."""
+    out = os.path.join(out_dir, f"liboracle_mutant{n}.so")
+    _build.build(out=out, mutant=n, force=True)
+    return Oracle(out)

@@ -1,0 +1,270 @@
+// attn_api.cu -- the C ABI declared in include/exact_attn.h.
+//
+// Argument checking, TMA tensor-map encoding and kernel launches. This is the
+// only translation unit of the library: the kernels live in the .cuh files it
+// includes, so the device status word below has a single definition.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "exact_attn.h"
+
+namespace eattn {
+// Device status word: kernels OR error bits into it; attn_status() reads and clears it.
+__device__ unsigned g_attn_status = 0;
+}  // namespace eattn
+
+#include "decode_sm100.cuh"
+#include "fwd_sm100.cuh"
+
+using namespace eattn;
+
+namespace {
+
+constexpr int kAbiVersion = 1;
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr long long kMaxSeq = 1ll << 30;
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn get_encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000,
+                                             cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    });
+    return fn;
+}
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+// Tensor map over a bf16 tensor viewed as [BH][N][D]; box = 128 rows x 64 columns,
+// 128-byte swizzle, out-of-range rows read as zero.
+bool encode_bf16_map(CUtensorMap* map, const void* base, int BH, int N, int D) {
+    EncodeTiledFn enc = get_encode_fn();
+    if (!enc) return false;
+    cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)N, (cuuint64_t)BH};
+    cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)N * D * 2};
+    cuuint32_t box[3] = {64, 128, 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims,
+                     strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                     CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+struct DeviceInfo {
+    int sms = 0;
+    bool fwd_attr_set[4] = {false, false, false, false};
+};
+DeviceInfo g_dev[64];
+std::mutex g_dev_mu;
+
+int current_device() {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return -1;
+    return dev;
+}
+
+template <int D, bool CAUSAL>
+attn_status_t launch_fwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                         const FwdParams& p, cudaStream_t stream) {
+    using T = FwdTraits<D>;
+    const int dev = current_device();
+    if (dev < 0 || dev >= 64) return ATTN_ERR_CUDA;
+    auto kern = attn_fwd_sm100_kernel<D, CAUSAL>;
+    int sms;
+    {
+        std::lock_guard<std::mutex> lk(g_dev_mu);
+        DeviceInfo& di = g_dev[dev];
+        if (di.sms == 0 &&
+            cudaDeviceGetAttribute(&di.sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+            return ATTN_ERR_CUDA;
+        const int slot = (D == 128 ? 2 : 0) + (CAUSAL ? 1 : 0);
+        if (!di.fwd_attr_set[slot]) {
+            if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     T::kSmemBytes) != cudaSuccess)
+                return ATTN_ERR_CUDA;
+            di.fwd_attr_set[slot] = true;
+        }
+        sms = di.sms;
+    }
+    const int grid = p.num_units < sms ? p.num_units : sms;
+    kern<<<grid, T::kThreads, T::kSmemBytes, stream>>>(tq, tk, tv, p);
+    return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+attn_status_t check_sizes(int B, int H, long long N1, long long N2) {
+    if (B < 1 || H < 1 || N1 < 1 || N2 < 1) return ATTN_ERR_INVALID_ARG;
+    if (N1 > kMaxSeq || N2 > kMaxSeq) return ATTN_ERR_INVALID_ARG;
+    if ((long long)B * H > (1ll << 24)) return ATTN_ERR_INVALID_ARG;
+    return ATTN_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int attn_abi_version(void) { return kAbiVersion; }
+
+const char* attn_strerror(attn_status_t s) {
+    switch (s) {
+        case ATTN_OK: return "ok";
+        case ATTN_ERR_INVALID_ARG: return "invalid argument (null pointer or bad size)";
+        case ATTN_ERR_UNSUPPORTED: return "unsupported configuration (head dim must be 64 or 128)";
+        case ATTN_ERR_ALIGNMENT: return "misaligned pointer (bf16 tensors need 16 bytes, fp32 4)";
+        case ATTN_ERR_CUDA: return "CUDA error while launching or running a kernel";
+        case ATTN_ERR_TIMEOUT: return "a kernel pipeline wait timed out; outputs are invalid";
+    }
+    return "unknown status";
+}
+
+attn_status_t attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B,
+                       int H, int Nq, int Nkv, int d, int causal, float scale, void* stream) {
+    if (!q || !k || !v || !o || !lse) return ATTN_ERR_INVALID_ARG;
+    if (causal != 0 && causal != 1) return ATTN_ERR_INVALID_ARG;
+    if (!(scale > 0.f) || !std::isfinite(scale)) return ATTN_ERR_INVALID_ARG;
+    attn_status_t s = check_sizes(B, H, Nq, Nkv);
+    if (s != ATTN_OK) return s;
+    if (d != 64 && d != 128) return ATTN_ERR_UNSUPPORTED;
+    if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) ||
+        !aligned(lse, 4))
+        return ATTN_ERR_ALIGNMENT;
+
+    const int BH = B * H;
+    CUtensorMap tq, tk, tv;
+    if (!encode_bf16_map(&tq, q, BH, Nq, d) || !encode_bf16_map(&tk, k, BH, Nkv, d) ||
+        !encode_bf16_map(&tv, v, BH, Nkv, d))
+        return ATTN_ERR_CUDA;
+    FwdParams p;
+    p.o = static_cast<uint16_t*>(o);
+    p.lse = lse;
+    p.BH = BH;
+    p.Nq = Nq;
+    p.Nkv = Nkv;
+    p.num_qb = (Nq + 255) / 256;
+    const long long units = (long long)BH * p.num_qb;
+    if (units > (1ll << 30)) return ATTN_ERR_INVALID_ARG;
+    p.num_units = (int)units;
+    p.scale_log2 = scale * kLog2e;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (d == 128)
+        return causal ? launch_fwd<128, true>(tq, tk, tv, p, st)
+                      : launch_fwd<128, false>(tq, tk, tv, p, st);
+    return causal ? launch_fwd<64, true>(tq, tk, tv, p, st)
+                  : launch_fwd<64, false>(tq, tk, tv, p, st);
+}
+
+attn_status_t attn_decode_partials(const void* q, const void* k, const void* v, float* o_part,
+                                   float* lse_part, int B, int H, int Nkv, int d, float scale,
+                                   int num_splits, void* stream) {
+    if (!q || !k || !v || !o_part || !lse_part) return ATTN_ERR_INVALID_ARG;
+    if (!(scale > 0.f) || !std::isfinite(scale)) return ATTN_ERR_INVALID_ARG;
+    attn_status_t s = check_sizes(B, H, Nkv, 1);
+    if (s != ATTN_OK) return s;
+    if (num_splits < 1 || num_splits > 65535) return ATTN_ERR_INVALID_ARG;
+    if (d != 64 && d != 128) return ATTN_ERR_UNSUPPORTED;
+    if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o_part, 4) ||
+        !aligned(lse_part, 4))
+        return ATTN_ERR_ALIGNMENT;
+    DecodeParams p;
+    p.q = static_cast<const uint16_t*>(q);
+    p.k = static_cast<const uint16_t*>(k);
+    p.v = static_cast<const uint16_t*>(v);
+    p.o_part = o_part;
+    p.lse_part = lse_part;
+    p.Nkv = Nkv;
+    p.S = num_splits;
+    p.L = (int)(((long long)Nkv + num_splits - 1) / num_splits);
+    p.scale_log2 = scale * kLog2e;
+    dim3 grid(num_splits, B * H);
+    if (B * H > 65535) return ATTN_ERR_INVALID_ARG;   // grid.y limit
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (d == 128)
+        attn_decode_partials_kernel<128><<<grid, DecodeTraits<128>::kThreads, 0, st>>>(p);
+    else
+        attn_decode_partials_kernel<64><<<grid, DecodeTraits<64>::kThreads, 0, st>>>(p);
+    return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+attn_status_t attn_lse_merge(const float* o_part, const float* lse_part, void* o, float* lse,
+                             int B, int H, int S, int d, void* stream) {
+    if (!o_part || !lse_part || !o || !lse) return ATTN_ERR_INVALID_ARG;
+    attn_status_t s = check_sizes(B, H, 1, 1);
+    if (s != ATTN_OK) return s;
+    if (S < 1 || S > 65535) return ATTN_ERR_INVALID_ARG;
+    if (d != 64 && d != 128) return ATTN_ERR_UNSUPPORTED;
+    if (!aligned(o_part, 4) || !aligned(lse_part, 4) || !aligned(o, 2) || !aligned(lse, 4))
+        return ATTN_ERR_ALIGNMENT;
+    const int BH = B * H;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (d == 128)
+        attn_lse_merge_kernel<128><<<BH, 128, 0, st>>>(o_part, lse_part,
+                                                       static_cast<uint16_t*>(o), lse, S);
+    else
+        attn_lse_merge_kernel<64><<<BH, 64, 0, st>>>(o_part, lse_part,
+                                                     static_cast<uint16_t*>(o), lse, S);
+    return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+size_t attn_decode_workspace_bytes(int B, int H, int d, int num_splits) {
+    if (B < 1 || H < 1 || num_splits < 1 || (d != 64 && d != 128)) return 0;
+    const size_t bhs = (size_t)B * H * num_splits;
+    const size_t o_bytes = (bhs * d * 4 + 255) / 256 * 256;
+    const size_t l_bytes = (bhs * 4 + 255) / 256 * 256;
+    return o_bytes + l_bytes;
+}
+
+attn_status_t attn_decode_splitkv(const void* q, const void* k, const void* v, void* o,
+                                  float* lse, int B, int H, int Nkv, int d, float scale,
+                                  int num_splits, void* workspace, size_t workspace_bytes,
+                                  void* stream) {
+    if (!workspace) return ATTN_ERR_INVALID_ARG;
+    const size_t need = attn_decode_workspace_bytes(B, H, d, num_splits);
+    if (need == 0) {
+        if (d != 64 && d != 128 && B >= 1 && H >= 1 && num_splits >= 1)
+            return ATTN_ERR_UNSUPPORTED;
+        return ATTN_ERR_INVALID_ARG;
+    }
+    if (workspace_bytes < need) return ATTN_ERR_INVALID_ARG;
+    if (!aligned(workspace, 256)) return ATTN_ERR_ALIGNMENT;
+    if (!o || !lse) return ATTN_ERR_INVALID_ARG;
+    if (!aligned(o, 2) || !aligned(lse, 4)) return ATTN_ERR_ALIGNMENT;
+    float* o_part = static_cast<float*>(workspace);
+    const size_t o_bytes = ((size_t)B * H * num_splits * d * 4 + 255) / 256 * 256;
+    float* lse_part = reinterpret_cast<float*>(static_cast<char*>(workspace) + o_bytes);
+    attn_status_t s = attn_decode_partials(q, k, v, o_part, lse_part, B, H, Nkv, d, scale,
+                                           num_splits, stream);
+    if (s != ATTN_OK) return s;
+    return attn_lse_merge(o_part, lse_part, o, lse, B, H, num_splits, d, stream);
+}
+
+attn_status_t attn_status(void* stream) {
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (cudaStreamSynchronize(st) != cudaSuccess) return ATTN_ERR_CUDA;
+    unsigned word = 0;
+    if (cudaMemcpyFromSymbol(&word, g_attn_status, sizeof(word)) != cudaSuccess)
+        return ATTN_ERR_CUDA;
+    if (word != 0) {
+        const unsigned zero = 0;
+        if (cudaMemcpyToSymbol(g_attn_status, &zero, sizeof(zero)) != cudaSuccess)
+            return ATTN_ERR_CUDA;
+    }
+    if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
+    return (word & kDevErrTimeout) ? ATTN_ERR_TIMEOUT : ATTN_OK;
+}
+
+}  // extern "C"

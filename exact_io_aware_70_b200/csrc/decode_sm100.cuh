@@ -1,0 +1,288 @@
+// decode_sm100.cuh -- split-KV decode for one query row per (batch, head).
+//
+// The decode method of "Describe Flash Attention at a high level"
+// (mantramindai), "Follow-up questions to expect", last question: with a single
+// query row there is no parallelism across query tiles, so the KV sequence is
+// split across thread blocks, each block computes the attention of the row
+// over its chunk of keys, and the partial results are merged with the same
+// max-and-sum trick the online softmax uses.
+//
+// With one query row the work is about one multiply-add per byte of K and V,
+// so it is bound by HBM bandwidth, not by the tensor cores: the partial kernel
+// streams K and V once with 16-byte non-caching loads, many in flight per
+// thread, and does the dot products and the P.V accumulation on the fp32 CUDA
+// cores. Within a chunk it walks sub-blocks of kSub keys with the online
+// softmax (running max, running sum, rescaled accumulator).
+#pragma once
+
+#include <cstdint>
+
+#include "ptx_sm100.cuh"
+
+namespace eattn {
+
+struct DecodeParams {
+    const uint16_t* q;   // bf16 [BH, D]
+    const uint16_t* k;   // bf16 [BH, Nkv, D]
+    const uint16_t* v;   // bf16 [BH, Nkv, D]
+    float* o_part;       // fp32 [BH, S, D]
+    float* lse_part;     // fp32 [BH, S]
+    int Nkv;
+    int S;               // number of chunks
+    int L;               // keys per chunk = ceil(Nkv / S)
+    float scale_log2;    // scale * log2(e)
+};
+
+__device__ __forceinline__ uint4 ld_stream_16B(const void* p) {
+    uint4 r;
+    asm volatile("ld.global.nc.L1::no_allocate.L2::256B.v4.u32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+                 : "l"(p));
+    return r;
+}
+
+// bf16 pair packed in a 32-bit word -> two fp32 (exact)
+__device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
+
+__device__ __forceinline__ float dot8(const uint4& kv, const float (&q)[8]) {
+    float a = bf16_lo(kv.x) * q[0];
+    a = fmaf(bf16_hi(kv.x), q[1], a);
+    a = fmaf(bf16_lo(kv.y), q[2], a);
+    a = fmaf(bf16_hi(kv.y), q[3], a);
+    a = fmaf(bf16_lo(kv.z), q[4], a);
+    a = fmaf(bf16_hi(kv.z), q[5], a);
+    a = fmaf(bf16_lo(kv.w), q[6], a);
+    a = fmaf(bf16_hi(kv.w), q[7], a);
+    return a;
+}
+
+__device__ __forceinline__ void axpy8(float p, const uint4& kv, float (&acc)[8]) {
+    acc[0] = fmaf(p, bf16_lo(kv.x), acc[0]);
+    acc[1] = fmaf(p, bf16_hi(kv.x), acc[1]);
+    acc[2] = fmaf(p, bf16_lo(kv.y), acc[2]);
+    acc[3] = fmaf(p, bf16_hi(kv.y), acc[3]);
+    acc[4] = fmaf(p, bf16_lo(kv.z), acc[4]);
+    acc[5] = fmaf(p, bf16_hi(kv.z), acc[5]);
+    acc[6] = fmaf(p, bf16_lo(kv.w), acc[6]);
+    acc[7] = fmaf(p, bf16_hi(kv.w), acc[7]);
+}
+
+template <int D>
+struct DecodeTraits {
+    static constexpr int kThreads = 256;
+    static constexpr int kLanesPerRow = D / 8;                     // 16-byte pieces per row
+    static constexpr int kRowsPerPass = kThreads / kLanesPerRow;   // rows covered by one load of all threads
+    static constexpr int kBatch = 8;                               // rows in flight per thread
+    static constexpr int kSub = kRowsPerPass * kBatch * 4;         // keys per sub-block
+};
+
+// Sum 8 per-lane partial values over the kLanes lanes of a row group so that
+// each lane ends with one complete sum: a transpose-reduce (each exchange step
+// halves the number of values a lane carries). On return, lane l of the group
+// holds the sum for value index ((l >> 1) & 7) when kLanes == 16, or (l & 7)
+// when kLanes == 8.
+template <int kLanes>
+__device__ __forceinline__ float group_transpose_reduce8(float (&v)[8], int lane) {
+    // step: 8 values -> 4
+    {
+        constexpr int off = kLanes / 2;
+        const bool hi = (lane & off) != 0;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const float send = hi ? v[i] : v[i + 4];
+            const float keep = hi ? v[i + 4] : v[i];
+            v[i] = keep + __shfl_xor_sync(0xffffffffu, send, off);
+        }
+    }
+    // 4 -> 2
+    {
+        constexpr int off = kLanes / 4;
+        const bool hi = (lane & off) != 0;
+#pragma unroll
+        for (int i = 0; i < 2; ++i) {
+            const float send = hi ? v[i] : v[i + 2];
+            const float keep = hi ? v[i + 2] : v[i];
+            v[i] = keep + __shfl_xor_sync(0xffffffffu, send, off);
+        }
+    }
+    // 2 -> 1
+    {
+        constexpr int off = kLanes / 8;
+        const bool hi = (lane & off) != 0;
+        const float send = hi ? v[0] : v[1];
+        const float keep = hi ? v[1] : v[0];
+        v[0] = keep + __shfl_xor_sync(0xffffffffu, send, off);
+    }
+    if (kLanes == 16) v[0] += __shfl_xor_sync(0xffffffffu, v[0], 1);
+    return v[0];
+}
+
+template <int D>
+__device__ __forceinline__ int reduce_owner_index(int glane) {
+    // which of the 8 values a lane of its row group ends up holding
+    return DecodeTraits<D>::kLanesPerRow == 16
+               ? ((glane >> 3) & 1) * 4 + ((glane >> 2) & 1) * 2 + ((glane >> 1) & 1)
+               : ((glane >> 2) & 1) * 4 + ((glane >> 1) & 1) * 2 + (glane & 1);
+}
+
+template <int D>
+__global__ void __launch_bounds__(256)
+    attn_decode_partials_kernel(const DecodeParams p) {
+    using T = DecodeTraits<D>;
+    constexpr int LPR = T::kLanesPerRow, RPP = T::kRowsPerPass, NB = T::kBatch;
+    constexpr int SUB = T::kSub;
+    __shared__ float s_score[SUB];
+    __shared__ float s_red[32];
+    __shared__ float s_acc[RPP][D + 4];
+
+    const int c = blockIdx.x;            // chunk
+    const int bh = blockIdx.y;
+    const int tid = threadIdx.x;
+    const int lane = tid & 31, warp = tid >> 5;
+    const int cc = tid % LPR;            // which 16-byte piece of a row
+    const int rs = tid / LPR;            // row slot within a pass
+    const int glane = tid % LPR;         // lane within the row group
+
+    const long long j0 = (long long)c * p.L;
+    const long long j1 = min(j0 + (long long)p.L, (long long)p.Nkv);
+    const int n = j1 > j0 ? (int)(j1 - j0) : 0;
+    float* o_out = p.o_part + ((size_t)bh * p.S + c) * D;
+
+    if (n == 0) {   // empty chunk: weight zero in the merge
+        for (int x = tid; x < D; x += blockDim.x) o_out[x] = 0.f;
+        if (tid == 0) p.lse_part[(size_t)bh * p.S + c] = -INFINITY;
+        return;
+    }
+
+    // this thread's 8 query elements, pre-scaled so scores come out in log2 units
+    float qv[8];
+    {
+        const uint4 qq = *reinterpret_cast<const uint4*>(p.q + (size_t)bh * D + cc * 8);
+        const float s = p.scale_log2;
+        qv[0] = bf16_lo(qq.x) * s; qv[1] = bf16_hi(qq.x) * s;
+        qv[2] = bf16_lo(qq.y) * s; qv[3] = bf16_hi(qq.y) * s;
+        qv[4] = bf16_lo(qq.z) * s; qv[5] = bf16_hi(qq.z) * s;
+        qv[6] = bf16_lo(qq.w) * s; qv[7] = bf16_hi(qq.w) * s;
+    }
+    const uint16_t* kbase = p.k + ((size_t)bh * p.Nkv + j0) * D + cc * 8;
+    const uint16_t* vbase = p.v + ((size_t)bh * p.Nkv + j0) * D + cc * 8;
+
+    float m_run = -INFINITY, l_run = 0.f;
+    float acc[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) acc[i] = 0.f;
+
+    for (int sb = 0; sb < n; sb += SUB) {
+        const int nsub = min(SUB, n - sb);
+        // ---- scores for this sub-block: s_i = (scale*log2e) q . k_i
+        for (int base = 0; base < SUB; base += RPP * NB) {
+            uint4 kr[NB];
+#pragma unroll
+            for (int b = 0; b < NB; ++b) {
+                const int i = base + rs + RPP * b;
+                kr[b] = i < nsub ? ld_stream_16B(kbase + (size_t)(sb + i) * D)
+                                 : make_uint4(0, 0, 0, 0);
+            }
+            float part[8];
+#pragma unroll
+            for (int b = 0; b < NB; ++b) part[b] = dot8(kr[b], qv);
+            const float sum = group_transpose_reduce8<LPR>(part, glane);
+            const int owner = reduce_owner_index<D>(glane);
+            const bool writer = (LPR == 16) ? ((glane & 1) == 0) : true;
+            if (writer) {
+                const int i = base + rs + RPP * owner;
+                s_score[i] = i < nsub ? sum : -INFINITY;
+            }
+        }
+        __syncthreads();
+        // ---- sub-block max
+        float mx = -INFINITY;
+        for (int i = tid; i < SUB; i += blockDim.x) mx = fmaxf(mx, s_score[i]);
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+        if (lane == 0) s_red[warp] = mx;
+        __syncthreads();
+        mx = s_red[0];
+#pragma unroll
+        for (int w = 1; w < 8; ++w) mx = fmaxf(mx, s_red[w]);
+        const float m_new = fmaxf(m_run, mx);   // finite: the sub-block has >= 1 key
+        const float alpha = fast_exp2(m_run - m_new);   // 0 on the first sub-block
+        // ---- probabilities (unnormalised) and their sum
+        float ls = 0.f;
+        for (int i = tid; i < SUB; i += blockDim.x) {
+            const float e = fast_exp2(s_score[i] - m_new);
+            s_score[i] = e;
+            ls += e;
+        }
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) ls += __shfl_xor_sync(0xffffffffu, ls, off);
+        __syncthreads();                 // all reads of s_red (max) done
+        if (lane == 0) s_red[warp] = ls;
+        __syncthreads();
+        float lsum = 0.f;
+#pragma unroll
+        for (int w = 0; w < 8; ++w) lsum += s_red[w];
+        l_run = l_run * alpha + lsum;
+        m_run = m_new;
+        // ---- accumulate P.V for this thread's 8 columns
+#pragma unroll
+        for (int i = 0; i < 8; ++i) acc[i] *= alpha;
+        for (int base = 0; base < SUB; base += RPP * NB) {
+            uint4 vr[NB];
+#pragma unroll
+            for (int b = 0; b < NB; ++b) {
+                const int i = base + rs + RPP * b;
+                vr[b] = i < nsub ? ld_stream_16B(vbase + (size_t)(sb + i) * D)
+                                 : make_uint4(0, 0, 0, 0);
+            }
+#pragma unroll
+            for (int b = 0; b < NB; ++b) axpy8(s_score[base + rs + RPP * b], vr[b], acc);
+        }
+        __syncthreads();                 // s_score and s_red are reused next sub-block
+    }
+    // ---- combine the RPP row slots, normalise, write the partial
+#pragma unroll
+    for (int i = 0; i < 8; ++i) s_acc[rs][cc * 8 + i] = acc[i];
+    __syncthreads();
+    const float inv = 1.0f / l_run;
+    for (int x = tid; x < D; x += blockDim.x) {
+        float s = 0.f;
+#pragma unroll 4
+        for (int r = 0; r < RPP; ++r) s += s_acc[r][x];
+        o_out[x] = s * inv;
+    }
+    if (tid == 0)
+        p.lse_part[(size_t)bh * p.S + c] = (m_run + log2f(l_run)) * 0.69314718055994531f;
+}
+
+// ------------------------------------------------------------------ merge --
+// One block of D threads per (batch, head): thread x owns output column x.
+//   M = max_c lse_c;  w_c = exp(lse_c - M);  LSE = M + ln sum_c w_c;
+//   O = sum_c w_c O_c / sum_c w_c.
+template <int D>
+__global__ void __launch_bounds__(D)
+    attn_lse_merge_kernel(const float* __restrict__ o_part, const float* __restrict__ lse_part,
+                          uint16_t* __restrict__ o, float* __restrict__ lse, int S) {
+    const int bh = blockIdx.x;
+    const int x = threadIdx.x;
+    const float* lp = lse_part + (size_t)bh * S;
+    const float* op = o_part + (size_t)bh * S * D + x;
+    float M = -INFINITY;
+    for (int c = 0; c < S; ++c) M = fmaxf(M, lp[c]);
+    float W = 0.f, acc = 0.f;
+    if (M != -INFINITY) {
+        constexpr float kLog2e = 1.4426950408889634f;
+        for (int c = 0; c < S; ++c) {
+            const float w = fast_exp2((lp[c] - M) * kLog2e);
+            W += w;
+            acc = fmaf(w, op[(size_t)c * D], acc);
+        }
+    }
+    const float out = W > 0.f ? acc / W : 0.f;
+    const uint32_t packed = pack_bf16x2(out, 0.f);
+    o[(size_t)bh * D + x] = (uint16_t)(packed & 0xFFFFu);
+    if (x == 0) lse[bh] = W > 0.f ? M + logf(W) : -INFINITY;
+}
+
+}  // namespace eattn

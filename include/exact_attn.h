@@ -1,0 +1,152 @@
+/*
+ * exact_attn.h -- C ABI of the B200 (sm_100a) exact-attention library.
+ *
+ * The library computes exact scaled-dot-product attention the IO-aware way:
+ *   O = softmax(scale * Q K^T [+ causal mask]) V,   LSE_i = ln sum_j exp(scale * q_i . k_j)
+ * with Q/K/V tiles staged on chip and the score and probability matrices never
+ * written to device memory, as described in "Describe Flash Attention at a
+ * high level" (mantramindai), section "The two ideas" (tiling and online
+ * softmax), and "How FlashAttention Speeds Up the Attention Layer"
+ * (hassanahmed.net), the tiling and online-softmax paragraphs. The result is
+ * the same as the plain definition up to floating-point rounding
+ * (mantramindai, "Follow-up questions to expect", first question).
+ *
+ * Conventions for every entry point:
+ *   - All tensor pointers are DEVICE pointers owned by the caller. The library
+ *     never allocates, frees or keeps them past the call.
+ *   - Tensors are dense and row-major: Q, O are [B, H, Nq, d]; K, V are
+ *     [B, H, Nkv, d]; LSE is [B, H, Nq]. Q, K, V, O are bfloat16 (passed as
+ *     void*); LSE and split partials are fp32.
+ *   - Every call is asynchronous on `stream` (a cudaStream_t passed as void*;
+ *     NULL means the legacy default stream). It returns after enqueueing.
+ *   - Argument errors are reported synchronously, before anything is launched:
+ *     ATTN_ERR_INVALID_ARG (null pointer, non-positive size, size overflow),
+ *     ATTN_ERR_UNSUPPORTED (head dim other than 64 or 128), ATTN_ERR_ALIGNMENT
+ *     (a bf16 tensor not 16-byte aligned, an fp32 tensor not 4-byte aligned).
+ *     No silent fallback exists: an input the kernels do not handle is refused.
+ *   - Errors seen while launching return ATTN_ERR_CUDA. Errors inside a kernel
+ *     (a pipeline wait that gave up after its time limit) are recorded in a
+ *     device status word and reported by attn_status().
+ *   - Causal masking is bottom-right aligned: key j is visible to query i iff
+ *     j <= i + (Nkv - Nq). A query row with no visible key gets O = 0 and
+ *     LSE = -inf.
+ *   - LSE is the natural logarithm of the sum of exp over the visible scaled
+ *     scores.
+ */
+#ifndef EXACT_ATTN_B200_H
+#define EXACT_ATTN_B200_H
+
+#include <stddef.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    ATTN_OK = 0,
+    ATTN_ERR_INVALID_ARG = 1,
+    ATTN_ERR_UNSUPPORTED = 2,
+    ATTN_ERR_ALIGNMENT = 3,
+    ATTN_ERR_CUDA = 4,
+    ATTN_ERR_TIMEOUT = 5
+} attn_status_t;
+
+/* Version of this ABI (bumped on any incompatible change). */
+int attn_abi_version(void);
+
+/*
+ * Prefill forward: O and LSE for Nq query rows against Nkv keys per (b, h).
+ *
+ * Defines: the fused attention kernel of "flashattention-memory-bound"
+ * (appliedaiprep), "A strong answer" (QK^T, softmax and .V fused in one kernel,
+ * tiles kept on chip), with the online-softmax recurrence of mantramindai
+ * "The two ideas" (running max m and sum l; earlier partial output rescaled by
+ * exp(m_old - m_new)). The per-row LSE is emitted so that a later merge or a
+ * backward pass can use it.
+ *
+ *   q   bf16 [B, H, Nq, d]      (read)
+ *   k   bf16 [B, H, Nkv, d]     (read)
+ *   v   bf16 [B, H, Nkv, d]     (read)
+ *   o   bf16 [B, H, Nq, d]      (written; rounded to nearest even)
+ *   lse fp32 [B, H, Nq]         (written)
+ *   d in {64, 128}; B, H, Nq, Nkv >= 1; causal 0 or 1; scale finite (usually
+ *   1/sqrt(d)). Any Nq, Nkv is accepted; tails of a 128-row tile are masked.
+ */
+attn_status_t attn_fwd(const void *q, const void *k, const void *v, void *o, float *lse,
+                       int B, int H, int Nq, int Nkv, int d, int causal, float scale,
+                       void *stream);
+
+/*
+ * Split-KV decode, step 1: per-chunk partials for one query row per (b, h).
+ *
+ * Defines: the decode method of "Describe Flash Attention at a high level"
+ * (mantramindai), "Follow-up questions to expect", last question: with one
+ * query row, parallelism comes from splitting the KV sequence across thread
+ * blocks. The keys are cut into num_splits chunks of L = ceil(Nkv / num_splits)
+ * consecutive keys (the last chunk shorter; trailing chunks may be empty).
+ * Chunk c yields the exact attention of the row restricted to its keys,
+ * normalised within the chunk, and that chunk's LSE.
+ *
+ *   q        bf16 [B, H, 1, d]        (read)
+ *   k, v     bf16 [B, H, Nkv, d]      (read)
+ *   o_part   fp32 [B, H, num_splits, d]   (written; an empty chunk gives 0)
+ *   lse_part fp32 [B, H, num_splits]      (written; an empty chunk gives -inf)
+ *   d in {64, 128}; 1 <= num_splits <= 65535. No mask (decode sees every key).
+ */
+attn_status_t attn_decode_partials(const void *q, const void *k, const void *v,
+                                   float *o_part, float *lse_part, int B, int H, int Nkv,
+                                   int d, float scale, int num_splits, void *stream);
+
+/*
+ * Split-KV decode, step 2: merge per-chunk partials with the max-and-sum trick
+ * (mantramindai, "Follow-up questions to expect", last question):
+ *   M = max_c lse_c;  W = sum_c exp(lse_c - M);  LSE = M + ln W;
+ *   O = sum_c exp(lse_c - M) / W * O_c     (all chunks empty: O = 0, LSE = -inf)
+ *
+ *   o_part   fp32 [B, H, S, d]   (read)
+ *   lse_part fp32 [B, H, S]      (read)
+ *   o        bf16 [B, H, 1, d]   (written)
+ *   lse      fp32 [B, H, 1]      (written)
+ *   d in {64, 128}; 1 <= S <= 65535.
+ */
+attn_status_t attn_lse_merge(const float *o_part, const float *lse_part, void *o, float *lse,
+                             int B, int H, int S, int d, void *stream);
+
+/*
+ * Bytes of caller-provided workspace attn_decode_splitkv needs for the
+ * partials: B*H*num_splits*(d + 1)*4, rounded up to 256. Returns 0 for
+ * invalid sizes.
+ */
+size_t attn_decode_workspace_bytes(int B, int H, int d, int num_splits);
+
+/*
+ * Split-KV decode, both steps: attn_decode_partials into `workspace`, then
+ * attn_lse_merge into o and lse, enqueued in that order on `stream`.
+ *
+ *   workspace  device memory of at least attn_decode_workspace_bytes(...)
+ *              bytes, 256-byte aligned, owned by the caller; its contents on
+ *              entry do not matter and on return are unspecified. Two calls
+ *              that run at the same time must not share one workspace.
+ *   Other arguments as for attn_decode_partials and attn_lse_merge.
+ */
+attn_status_t attn_decode_splitkv(const void *q, const void *k, const void *v, void *o,
+                                  float *lse, int B, int H, int Nkv, int d, float scale,
+                                  int num_splits, void *workspace, size_t workspace_bytes,
+                                  void *stream);
+
+/*
+ * Synchronises `stream`, then returns and clears the device status word:
+ * ATTN_ERR_TIMEOUT if a kernel's pipeline wait gave up since the last call
+ * (its outputs are then invalid), ATTN_ERR_CUDA if the stream reported an
+ * error, ATTN_OK otherwise.
+ */
+attn_status_t attn_status(void *stream);
+
+/* A static, human-readable description of a status code. */
+const char *attn_strerror(attn_status_t status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* EXACT_ATTN_B200_H */

@@ -1,0 +1,104 @@
+"""The C-ABI library loads, exports every declared entry point, and rejects bad
+arguments before touching the GPU (so these run on a CPU-only host)."""
+import ctypes
+import importlib.util
+import os
+import re
+import shutil
+import sys
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "exact_attn.h")
+
+
+@pytest.fixture(scope="module")
+def ea():
+    from exact_io_aware_70_b200 import build
+    build.build()
+    import exact_io_aware_70_b200 as m
+    return m
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(attn_\w+)\s*\(", text)))
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for want in ("attn_fwd", "attn_decode_partials", "attn_lse_merge", "attn_decode_splitkv",
+                 "attn_decode_workspace_bytes", "attn_status", "attn_strerror",
+                 "attn_abi_version"):
+        assert want in names
+
+
+def test_library_exports_every_declared_symbol(ea):
+    lib = ctypes.CDLL(ea.LIB_PATH)
+    for name in declared_functions():
+        assert hasattr(lib, name), f"{name} declared in exact_attn.h but not exported"
+
+
+def test_version_and_strerror(ea):
+    assert ea.abi_version() == 1
+    for code in range(6):
+        assert ea.attn_strerror(code)
+    assert "unknown" in ea.attn_strerror(99)
+
+
+def test_fwd_rejects_bad_arguments_without_launching(ea):
+    L = ea.lib
+    p = 0x10000  # never dereferenced: every case below fails validation first
+    ok = dict(q=p, k=p, v=p, o=p, lse=p, B=1, H=1, Nq=128, Nkv=128, d=64, causal=0, scale=0.125)
+
+    def call(**kw):
+        a = dict(ok, **kw)
+        return L.attn_fwd(a["q"], a["k"], a["v"], a["o"], a["lse"], a["B"], a["H"], a["Nq"],
+                          a["Nkv"], a["d"], a["causal"], a["scale"], None)
+
+    assert call(q=None) == ea.ATTN_ERR_INVALID_ARG
+    assert call(lse=None) == ea.ATTN_ERR_INVALID_ARG
+    assert call(B=0) == ea.ATTN_ERR_INVALID_ARG
+    assert call(Nq=0) == ea.ATTN_ERR_INVALID_ARG
+    assert call(Nkv=-5) == ea.ATTN_ERR_INVALID_ARG
+    assert call(causal=2) == ea.ATTN_ERR_INVALID_ARG
+    assert call(scale=0.0) == ea.ATTN_ERR_INVALID_ARG
+    assert call(scale=float("nan")) == ea.ATTN_ERR_INVALID_ARG
+    assert call(d=96) == ea.ATTN_ERR_UNSUPPORTED
+    assert call(d=256) == ea.ATTN_ERR_UNSUPPORTED
+    assert call(q=p + 8) == ea.ATTN_ERR_ALIGNMENT
+    assert call(o=p + 2) == ea.ATTN_ERR_ALIGNMENT
+    assert call(lse=p + 2) == ea.ATTN_ERR_ALIGNMENT
+
+
+def test_decode_and_merge_reject_bad_arguments(ea):
+    L = ea.lib
+    p = 0x10000
+    assert L.attn_decode_partials(None, p, p, p, p, 1, 1, 64, 128, 0.1, 4, None) == 1
+    assert L.attn_decode_partials(p, p, p, p, p, 1, 1, 64, 128, 0.1, 0, None) == 1
+    assert L.attn_decode_partials(p, p, p, p, p, 1, 1, 64, 80, 0.1, 4, None) == 2
+    assert L.attn_decode_partials(p, p + 4, p, p, p, 1, 1, 64, 128, 0.1, 4, None) == 3
+    assert L.attn_lse_merge(p, p, p, p, 1, 1, 0, 128, None) == 1
+    assert L.attn_lse_merge(p, p, p, p, 1, 1, 4, 32, None) == 2
+    assert L.attn_lse_merge(p, p + 1, p, p, 1, 1, 4, 128, None) == 3
+    need = ea.attn_decode_workspace_bytes(2, 3, 128, 8)
+    assert need == ((2 * 3 * 8 * 128 * 4 + 255) // 256 + (2 * 3 * 8 * 4 + 255) // 256) * 256
+    assert ea.attn_decode_workspace_bytes(2, 3, 96, 8) == 0
+    assert L.attn_decode_splitkv(p, p, p, p, p, 2, 3, 64, 128, 0.1, 8, p, need - 1, None) == 1
+    assert L.attn_decode_splitkv(p, p, p, p, p, 2, 3, 64, 128, 0.1, 8, p + 16, need, None) == 3
+    assert L.attn_decode_splitkv(p, p, p, p, p, 2, 3, 64, 96, 0.1, 8, p, need, None) == 2
+
+
+def test_package_fails_loudly_without_the_library(tmp_path):
+    """No silent fallback: the binding refuses to import when the .so is absent."""
+    src = os.path.join(ROOT, "exact_io_aware_70_b200", "__init__.py")
+    pkg = tmp_path / "fake_pkg"
+    pkg.mkdir()
+    shutil.copy(src, pkg / "__init__.py")
+    spec = importlib.util.spec_from_file_location("fake_pkg", pkg / "__init__.py")
+    mod = importlib.util.module_from_spec(spec)
+    with pytest.raises(ImportError, match="missing"):
+        spec.loader.exec_module(mod)
+    sys.modules.pop("fake_pkg", None)

@@ -1,0 +1,546 @@
+#!/usr/bin/env python3
+"""Benchmark of the exact-attention hot path on B200.
+
+One step = one pass of the whole hot path over one batch of synthetic inputs:
+  * prefill forward on the 8192-token workload (B=1, H=32, N=8192, d=128,
+    causal), O and LSE  -> attn fwd TFLOP/s (the line's ``value``);
+  * split-KV decode on the 32K-cache workload (B=16, H=32, Nkv=32768, d=128,
+    64 chunks), partials + merge -> decode KV GB/s (``decode``).
+Inputs are seeded i.i.d. N(0,1) bf16 (seeded_inputs.py), resident in HBM
+before timing; they exceed the 126 MB L2 (192 MB prefill + 8.6 GB decode), so
+no extra flush is needed between steps.
+
+``--impl reference`` times the fp64 CPU oracle on a bounded sample of the same
+workloads instead (the reference arm); it never touches the GPU path.
+
+Multi-GPU (torchrun): every rank runs the same step on its own batch (seed +
+rank); the path has no data exchange, so scaling is weak and timings are the
+max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from seeded_inputs import WORKLOADS, make_workload  # noqa: E402
+
+METRIC = "attn fwd TFLOP/s & % BF16 tensor peak; decode KV GB/s & % HBM peak"
+PREFILL = WORKLOADS["prefill_8k"]
+DECODE = WORKLOADS["decode_32k"]
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as fh:
+            p = json.load(fh)
+        return {"hbm_gbs": float(p["hbm_gbs"]), "bf16_tflops": float(p["bf16_tflops"]),
+                "bf16_tflops_sustained": float(p["bf16_tflops_sustained"]), "source": "measured"}
+    except (OSError, KeyError, ValueError):
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+                "source": "fallback"}
+
+
+# --------------------------------------------------------------- work model --
+def prefill_pairs(w):
+    if w.causal:   # bottom-right aligned visible pairs
+        tot = 0
+        off = w.Nkv - w.Nq
+        # rows i see min(Nkv, max(0, i + off + 1)) keys
+        for i in range(w.Nq):
+            tot += min(w.Nkv, max(0, i + off + 1))
+        return tot
+    return w.Nq * w.Nkv
+
+
+def prefill_flops(w):
+    return 4.0 * w.d * w.B * w.H * prefill_pairs(w)
+
+
+def prefill_bytes(w):
+    return w.B * w.H * (2 * w.Nq * w.d * 2 + 2 * w.Nkv * w.d * 2 + 4 * w.Nq)
+
+
+def decode_kv_bytes(w):
+    return 2.0 * w.B * w.H * w.Nkv * w.d * 2
+
+
+def decode_partial_bytes(w):
+    """Compulsory traffic of the partial kernel: q, K, V read; partials written."""
+    return decode_kv_bytes(w) + w.B * w.H * (w.d * 2 + w.num_splits * (w.d + 1) * 4)
+
+
+def merge_bytes(w):
+    return w.B * w.H * (w.num_splits * (w.d + 1) * 4 + w.d * 2 + 4)
+
+
+# ---------------------------------------------------------------- helpers --
+def dist_env():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled while the timed region runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *exc):
+        self.lines = []
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                out, _ = self.proc.communicate()
+            self.lines = [ln for ln in out.splitlines() if ln.strip()]
+        return False
+
+    def summary(self, max_mhz_default=1965.0):
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in getattr(self, "lines", []):
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx.append(float(parts[2]))
+            except ValueError:
+                continue
+            for nm, val in zip(names, parts[5:9]):
+                if val.lower() == "active":
+                    reasons.add(nm)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": max_mhz_default, "reasons": ["unsampled"],
+                    "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx) if mx else max_mhz_default,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def kernel_source_hash():
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "exact_io_aware_70_b200", "csrc")
+    for f in sorted(os.listdir(csrc)):
+        if f.endswith((".cu", ".cuh")):
+            with open(os.path.join(csrc, f), "rb") as fh:
+                h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic():
+    """Per-launch DRAM traffic from the committed ncu summary, if taken on this source."""
+    path = os.path.join(ROOT, "profiles", "dram_traffic.json")
+    try:
+        with open(path) as fh:
+            rec = json.load(fh)
+    except (OSError, ValueError):
+        return {}
+    if rec.get("source_hash") != kernel_source_hash():
+        return {}
+    return rec.get("per_launch_bytes", {})
+
+
+# ------------------------------------------------------------ CPU oracle --
+def oracle_prefill_sample(budget_s, max_rows=None, max_heads=4):
+    """Time the oracle on evenly spaced query rows of the prefill workload's heads.
+
+    The row count grows until one head's sample takes a quarter of the budget
+    (or covers every row); whole heads are then repeated while the budget lasts.
+    """
+    import numpy as np
+
+    import oracle
+    from seeded_inputs import bf16_bits, make_qkv
+    w = PREFILL
+    orc = oracle.get()
+    q, k, v = make_qkv(1, max_heads, w.Nq, w.Nkv, w.d, w.seed)   # CPU generator
+    hb = [(bf16_bits(q[0, h]), bf16_bits(k[0, h]), bf16_bits(v[0, h])) for h in range(max_heads)]
+    nrows = 64
+    while True:
+        rows = np.linspace(0, w.Nq - 1, nrows).astype(np.int64)
+        t0 = time.perf_counter()
+        orc.attn_rows_bf16(*hb[0], rows, w.causal, w.scale)
+        dt = time.perf_counter() - t0
+        if dt > budget_s / 4 or nrows >= w.Nq or (max_rows and nrows >= max_rows):
+            break
+        nrows = min(w.Nq, nrows * 4)
+    heads = 1
+    while heads < max_heads and dt * (heads + 1) / heads < budget_s:
+        t0 = time.perf_counter()
+        orc.attn_rows_bf16(*hb[heads], rows, w.causal, w.scale)
+        dt += time.perf_counter() - t0
+        heads += 1
+    flops = heads * sum(4.0 * w.d * min(w.Nkv, int(r) + 1 + (w.Nkv - w.Nq)) for r in rows)
+    return {"flops": flops, "seconds": dt, "rows": int(nrows), "heads": heads,
+            "cores": orc.num_threads()}
+
+
+def oracle_decode_sample(budget_s):
+    import oracle
+    from seeded_inputs import bf16_bits, make_qkv
+    w = DECODE
+    orc = oracle.get()
+    q, k, v = make_qkv(1, 2, 1, w.Nkv, w.d, w.seed)
+    heads = 0
+    t0 = time.perf_counter()
+    while True:
+        for h in range(2):
+            orc.attn_rows_bf16(bf16_bits(q[0, h]), bf16_bits(k[0, h]), bf16_bits(v[0, h]), [0],
+                               False, w.scale)
+            heads += 1
+        dt = time.perf_counter() - t0
+        if dt > budget_s or heads >= 64:
+            break
+    return {"bytes": heads * 2.0 * w.Nkv * w.d * 2, "seconds": dt, "heads": heads,
+            "cores": orc.num_threads()}
+
+
+def cpu_baseline(budget_s=8.0):
+    pf = oracle_prefill_sample(budget_s)
+    dc = oracle_decode_sample(budget_s / 4)
+    return {
+        "value": pf["flops"] / pf["seconds"] / 1e12, "unit": "TFLOP/s", "cores": pf["cores"],
+        "kind": "oracle",
+        "sample": (f"fp64 oracle, {pf['rows']} evenly spaced query rows of each of "
+                   f"{pf['heads']} heads of prefill_8k ({pf['flops'] / 1e9:.1f} GFLOP in {pf['seconds']:.2f} s); "
+                   f"decode: {dc['heads']} (b,h) rows of decode_32k "
+                   f"({dc['bytes'] / 1e9:.2f} GB of K/V in {dc['seconds']:.2f} s)"),
+        "decode": {"value": dc["bytes"] / dc["seconds"] / 1e9, "unit": "GB/s"},
+    }
+
+
+def run_reference(args):
+    """Reference arm: the oracle, as it stands, on bounded samples of the workload."""
+    ws, rank, _ = dist_env()
+    if rank != 0:
+        return 0
+    sizes = []
+    for _ in range(max(0, args.warmup)):
+        oracle_prefill_sample(1.0, max_rows=256, max_heads=1)
+    times = []
+    flops = 0.0
+    for _ in range(args.steps):
+        r = oracle_prefill_sample(1.0, max_rows=256, max_heads=1)
+        times.append(r["seconds"])
+        flops = r["flops"]
+        sizes.append(r["rows"])
+    dc = oracle_decode_sample(1.0)
+    value = flops / statistics.mean(times) / 1e12
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s",
+        "n_gpus": ws, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * statistics.mean(times), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": "prefill_8k (sampled rows) + decode_32k (sampled heads)",
+                   "B": PREFILL.B, "H": PREFILL.H, "N": PREFILL.Nq, "d": PREFILL.d,
+                   "causal": PREFILL.causal, "parallelism": "cpu"},
+        "decode": {"value": dc["bytes"] / dc["seconds"] / 1e9, "unit": "GB/s"},
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": r["cores"],
+                         "kind": "oracle",
+                         "sample": f"{sizes[-1]} evenly spaced rows of one prefill_8k head per step"},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ------------------------------------------------------------ GPU arm --
+def _maybe_batch(w, batch):
+    import dataclasses
+    return dataclasses.replace(w, B=batch) if batch else w
+
+
+def run_ours(args):
+    import dataclasses
+
+    import torch
+    import torch.distributed as dist
+
+    import exact_io_aware_70_b200 as ea
+
+    ws, rank, local = dist_env()
+    torch.cuda.set_device(local)
+    if ws > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    dev = torch.device("cuda", local)
+    stream = torch.cuda.current_stream()
+    sp = stream.cuda_stream
+    L = ea.lib
+
+    if args.workload == "step":
+        pw, dw = PREFILL, DECODE
+    elif args.workload in ("prefill_8k", "prefill_16k", "gpt2_1k", "tiny"):
+        pw, dw = WORKLOADS[args.workload], None
+    else:
+        pw, dw = None, WORKLOADS[args.workload]
+    pw = _maybe_batch(pw, args.batch) if pw else None
+    dw = _maybe_batch(dw, args.batch) if dw else None
+
+    # ---- inputs resident in HBM (seed offset per rank: each rank its own batch)
+    kernels = []
+    if pw:
+        pw_r = dataclasses.replace(pw, seed=pw.seed + 1000 * rank)
+        q, k, v = make_workload(pw_r, device="cuda")
+        o = torch.empty_like(q)
+        lse = torch.empty((pw.B, pw.H, pw.Nq), dtype=torch.float32, device=dev)
+
+        def launch_prefill():
+            return L.attn_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
+                              lse.data_ptr(), pw.B, pw.H, pw.Nq, pw.Nkv, pw.d, int(pw.causal),
+                              pw.scale, sp)
+        kernels.append(("attn_fwd_sm100", launch_prefill))
+    if dw:
+        dw_r = dataclasses.replace(dw, seed=dw.seed + 1000 * rank)
+        dq, dk, dv = make_workload(dw_r, device="cuda")
+        do = torch.empty_like(dq)
+        dlse = torch.empty((dw.B, dw.H, 1), dtype=torch.float32, device=dev)
+        S = dw.num_splits
+        work = torch.empty(ea.attn_decode_workspace_bytes(dw.B, dw.H, dw.d, S), dtype=torch.uint8,
+                           device=dev)
+        o_bytes = ((dw.B * dw.H * S * dw.d * 4 + 255) // 256) * 256
+        o_part = work.data_ptr()
+        lse_part = work.data_ptr() + o_bytes
+
+        def launch_partials():
+            return L.attn_decode_partials(dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), o_part,
+                                          lse_part, dw.B, dw.H, dw.Nkv, dw.d, dw.scale, S, sp)
+
+        def launch_merge():
+            return L.attn_lse_merge(o_part, lse_part, do.data_ptr(), dlse.data_ptr(), dw.B, dw.H,
+                                    S, dw.d, sp)
+        kernels += [("attn_decode_partials", launch_partials), ("attn_lse_merge", launch_merge)]
+    torch.cuda.synchronize()
+
+    def step(evs=None):
+        for i, (name, fn) in enumerate(kernels):
+            if evs is not None:
+                evs[i].record(stream)
+            rc = fn()
+            if rc != 0:
+                raise RuntimeError(f"{name}: {ea.attn_strerror(rc)}")
+        if evs is not None:
+            evs[len(kernels)].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    if ea.attn_status() != 0:
+        raise RuntimeError("device status reported an error during warm-up")
+
+    K = args.steps
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(len(kernels) + 1)]
+          for _ in range(K)]
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local) as clk:
+        if ws > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+        t_start.record(stream)
+        for s in range(K):
+            step(ev[s])
+        t_end.record(stream)
+        torch.cuda.synchronize()
+        if ws > 1:
+            dist.barrier()
+    if ea.attn_status() != 0:
+        raise RuntimeError("device status reported an error in the timed region")
+    total_ms = t_start.elapsed_time(t_end)
+    per_kernel_ms = [statistics.mean(ev[s][i].elapsed_time(ev[s][i + 1]) for s in range(K))
+                     for i in range(len(kernels))]
+    times = torch.tensor([total_ms] + per_kernel_ms, dtype=torch.float64, device=dev)
+    if ws > 1:
+        dist.all_reduce(times, op=dist.ReduceOp.MAX)
+    total_ms, *per_kernel_ms = times.tolist()
+    kms = dict(zip([n for n, _ in kernels], per_kernel_ms))
+
+    # ---- e2e: the same work through the public API from pinned host buffers
+    e2e = None
+    if not args.no_e2e:
+        h2d = d2h = 0
+        if pw:
+            hq, hk, hv = (t.cpu().pin_memory() for t in (q, k, v))
+            ho = torch.empty(o.shape, dtype=o.dtype, pin_memory=True)
+            hl = torch.empty(lse.shape, dtype=lse.dtype, pin_memory=True)
+            h2d += sum(t.numel() * t.element_size() for t in (hq, hk, hv))
+            d2h += sum(t.numel() * t.element_size() for t in (ho, hl))
+        if dw:
+            hdq, hdk, hdv = (t.cpu().pin_memory() for t in (dq, dk, dv))
+            hdo = torch.empty(do.shape, dtype=do.dtype, pin_memory=True)
+            hdl = torch.empty(dlse.shape, dtype=dlse.dtype, pin_memory=True)
+            h2d += sum(t.numel() * t.element_size() for t in (hdq, hdk, hdv))
+            d2h += sum(t.numel() * t.element_size() for t in (hdo, hdl))
+
+        def e2e_prefill():
+            q.copy_(hq, non_blocking=True)
+            k.copy_(hk, non_blocking=True)
+            v.copy_(hv, non_blocking=True)
+            ea.attn_fwd(q, k, v, o, lse, pw.causal, pw.scale)
+            ho.copy_(o, non_blocking=True)
+            hl.copy_(lse, non_blocking=True)
+
+        def e2e_decode():
+            dq.copy_(hdq, non_blocking=True)
+            dk.copy_(hdk, non_blocking=True)
+            dv.copy_(hdv, non_blocking=True)
+            ea.attn_decode_splitkv(dq, dk, dv, do, dlse, dw.scale, S, work)
+            hdo.copy_(do, non_blocking=True)
+            hdl.copy_(dlse, non_blocking=True)
+
+        parts = ([e2e_prefill] if pw else []) + ([e2e_decode] if dw else [])
+        for fn in parts:
+            fn()
+        torch.cuda.synchronize()
+        E = max(2, min(K, 3))
+        ep = [torch.cuda.Event(enable_timing=True) for _ in range(len(parts) + 1)]
+        acc = [0.0] * len(parts)
+        for _ in range(E):
+            for i, fn in enumerate(parts):
+                ep[i].record(stream)
+                fn()
+            ep[len(parts)].record(stream)
+            torch.cuda.synchronize()
+            for i in range(len(parts)):
+                acc[i] += ep[i].elapsed_time(ep[i + 1]) / E
+        et = torch.tensor(acc, dtype=torch.float64, device=dev)
+        if ws > 1:
+            dist.all_reduce(et, op=dist.ReduceOp.MAX)
+        acc = et.tolist()
+        if ea.attn_status() != 0:
+            raise RuntimeError("device status reported an error in the e2e region")
+        e2e = {"h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": sum(acc),
+               "steps": E,
+               "path": "pinned host -> copy -> attn_fwd / attn_decode_splitkv -> copy back, "
+                       "per step, CUDA events on the launching stream"}
+        if pw:
+            e2e["value"] = ws * prefill_flops(pw) / (acc[0] * 1e-3) / 1e12
+            e2e["unit"] = "TFLOP/s"
+        if dw:
+            dec = {"value": ws * decode_kv_bytes(dw) / (acc[-1] * 1e-3) / 1e9, "unit": "GB/s"}
+            if pw:
+                e2e["decode"] = dec
+            else:
+                e2e.update(dec)
+
+    if ws > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return 0
+
+    pk = peaks()
+    traffic = recorded_traffic()
+    step_ms = sum(per_kernel_ms)
+    roof = {}
+    if pw:
+        t = kms["attn_fwd_sm100"]
+        a = prefill_flops(pw) / (t * 1e-3) / 1e12
+        roof["attn_fwd_sm100"] = {
+            "bound": "tensor", "achieved": a, "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
+            "frac": a / pk["bf16_tflops"], "frac_of_sustained": a / pk["bf16_tflops_sustained"],
+            "traffic": traffic.get("attn_fwd_sm100"), "algorithmic_bytes": prefill_bytes(pw),
+            "algorithmic_flops": prefill_flops(pw), "ms": t, "share": t / step_ms}
+    if dw:
+        for name, nbytes in (("attn_decode_partials", decode_partial_bytes(dw)),
+                             ("attn_lse_merge", merge_bytes(dw))):
+            t = kms[name]
+            a = nbytes / (t * 1e-3) / 1e9
+            roof[name] = {"bound": "hbm", "achieved": a, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                          "frac": a / pk["hbm_gbs"], "traffic": traffic.get(name),
+                          "algorithmic_bytes": nbytes, "ms": t, "share": t / step_ms}
+    dominant = max(roof, key=lambda n: roof[n]["ms"])
+    dom = dict(roof[dominant], kernel=dominant)
+    cfg = {"workload": "prefill_8k + decode_32k" if args.workload == "step" else args.workload,
+           "l2": "inputs larger than L2 (126 MB); no flush" if not args.batch else
+                 "reduced batch for profiling",
+           "parallelism": f"replicas x{ws}" if ws > 1 else "1 GPU"}
+    line = {"metric": METRIC}
+    if pw:
+        pf = kms["attn_fwd_sm100"]
+        cfg["prefill"] = {"B": pw.B, "H": pw.H, "N": pw.Nq, "d": pw.d, "causal": pw.causal,
+                          "flop_per_step": prefill_flops(pw)}
+        line.update(value=ws * prefill_flops(pw) / (pf * 1e-3) / 1e12, unit="TFLOP/s")
+        line["prefill"] = {"value": line["value"], "unit": "TFLOP/s", "ms": pf,
+                           "frac_of_bf16_peak": roof["attn_fwd_sm100"]["frac"]}
+    if dw:
+        dms = kms["attn_decode_partials"] + kms["attn_lse_merge"]
+        cfg["decode"] = {"B": dw.B, "H": dw.H, "Nkv": dw.Nkv, "d": dw.d, "splits": dw.num_splits,
+                         "kv_bytes_per_step": decode_kv_bytes(dw)}
+        dgbs = decode_kv_bytes(dw) / (dms * 1e-3) / 1e9
+        line["decode"] = {"value": ws * dgbs, "unit": "GB/s", "ms": dms,
+                          "frac_of_hbm_peak": dgbs / pk["hbm_gbs"]}
+        if not pw:
+            line.update(value=ws * dgbs, unit="GB/s")
+    line.update({
+        "n_gpus": ws, "steps": K, "warmup": args.warmup, "ms_per_step": total_ms / K,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic", "config": cfg, "roofline": dom, "roofline_kernels": roof,
+        "peaks": dict(pk, note="of measured" if pk["source"] == "measured" else "of fallback"),
+        "clocks": clk.summary(max_mhz_default=1965.0),
+        "gpu_launches": len(kernels) * K, "e2e": e2e,
+    })
+    if ws == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(args.cpu_budget)
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__.splitlines()[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="step",
+                    choices=["step", "prefill_8k", "prefill_16k", "gpt2_1k", "tiny", "decode_32k"],
+                    help="step = prefill_8k + decode_32k (the default bench line)")
+    ap.add_argument("--batch", type=int, default=0,
+                    help="override the batch size (small profiling captures only)")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-budget", type=float, default=8.0,
+                    help="seconds of oracle work for the CPU baseline")
+    args = ap.parse_args()
+    if args.warmup < 3 and args.impl == "ours":
+        args.warmup = 3
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -6,6 +6,7 @@ nvcc for sm_100a only. No GPU is needed to build.
 from __future__ import annotations
 
 import os
+import re
 import subprocess
 import sys
 
@@ -47,7 +48,35 @@ def build(force: bool = False, verbose: bool = False) -> str:
         raise RuntimeError("nvcc failed building the attention library")
     if verbose:
         sys.stderr.write(res.stderr)
+    check_register_budget(res.stdout + res.stderr)
     return LIB
+
+
+# The prefill kernel redistributes registers with setmaxnreg assuming each of
+# its 384 threads received exactly this many at launch (FwdTraits::kLaunchRegs).
+# Fewer at launch would make the softmax warpgroups' increase wait forever, so
+# the build refuses to produce such a library.
+FWD_LAUNCH_REGS = 168
+
+
+def check_register_budget(ptxas_log: str) -> None:
+    current = None
+    seen = 0
+    for line in ptxas_log.splitlines():
+        m = re.search(r"Compiling entry function '([^']+)'", line)
+        if m:
+            current = m.group(1)
+            continue
+        m = re.search(r"Used (\d+) registers", line)
+        if m and current and "attn_fwd_sm100_kernel" in current:
+            seen += 1
+            if int(m.group(1)) != FWD_LAUNCH_REGS:
+                os.remove(LIB)
+                raise RuntimeError(f"{current} uses {m.group(1)} registers, expected "
+                                   f"{FWD_LAUNCH_REGS}: the setmaxnreg split would not fit")
+    if seen == 0:
+        os.remove(LIB)
+        raise RuntimeError("ptxas register report for the prefill kernel not found")
 
 
 if __name__ == "__main__":

@@ -14,14 +14,19 @@
 // How it maps onto a B200 SM (this design is ours; the pages' A100/H100
 // kernels are prior art only):
 //   * Persistent grid, one CTA per SM. A work unit is (batch*head, 256 query
-//     rows) = two 128-row Q tiles; units are handed out heaviest-first so the
-//     causal triangle balances across the 148 SMs.
+//     rows) = two 128-row Q tiles. Units are sorted heaviest-first and dealt
+//     to the CTAs in alternating direction each round (CTA i takes unit
+//     r*G + i in even rounds, r*G + G-1-i in odd rounds), which balances the
+//     causal triangle across the 148 SMs about as well as longest-first greedy.
 //   * Warp 8 (one elected lane) is the TMA producer: Q tiles once per unit,
 //     then K_j and V_j tiles into a ring of shared-memory slots, 128-byte
 //     swizzled, completion counted on mbarriers.
 //   * Warp 9 (one elected lane) issues every tcgen05.mma: S_t = Q_t K_j^T into
 //     tensor memory (fp32, 128x128), and O_t += P_t V_j with P_t read straight
 //     from tensor memory (bf16, aliased over S_t's first 64 columns).
+//   * 384 threads = 3 warpgroups; warps 10-11 only complete the third
+//     warpgroup so it can shrink its register budget (setmaxnreg) in favour
+//     of the two softmax warpgroups.
 //   * Warps 0-3 and 4-7 are the softmax groups of Q tile 0 and Q tile 1, one
 //     thread per query row (= TMEM lane). While one group exponentiates its
 //     tile, the tensor core works on the other tile's products (ping-pong).
@@ -29,7 +34,19 @@
 //     grows by more than 2^8 (lazy rescaling: exact, since every p and l uses
 //     the same stale reference max), and runs the epilogue (O / l -> bf16,
 //     LSE = ln 2 * (m + log2 l)).
-//   * Exponentials are base 2 with log2(e) folded into the scale.
+//   * Exponentials are base 2 with log2(e) folded into the scale, computed
+//     with MUFU ex2 on pairs prepared by sm_100's packed f32x2 FMA; the row
+//     max uses the three-input max. Optionally (EATTN_POLY_EVERY = k > 0) one
+//     pair in every k is exponentiated on the FMA pipe (exp2_poly_pair)
+//     instead; measured on B200 this is slower at every k tried (2, 3, 4, 8)
+//     because the softmax is issue-bound rather than MUFU-bound once the
+//     pairs are packed, so it is off by default. A masked (-inf) score comes
+//     out of the polynomial as about 2^-125 rather than 0: negligible next to
+//     the row sum (at least 1 once a row has seen a visible key), and rows with
+//     no visible key at all are set to O = 0, LSE = -inf in the epilogue.
+//   * P_t is handed to the MMA warp in two halves (keys 0-63, then 64-127),
+//     so the first half of O_t += P_t V_j runs while the second half of the
+//     exponentials is still being computed.
 //   * Tensor memory columns: S0 [0,128), S1 [128,256), O0 [256,256+d),
 //     O1 [256+d, 256+2d).
 #pragma once
@@ -61,13 +78,38 @@ struct FwdTraits {
     static constexpr int kPanels = D / 64;
     static constexpr int kTileBytes = kPanels * kPanelBytes;
     static constexpr int kSlots = (D == 128) ? 4 : 8;     // K/V ring depth (tiles)
-    static constexpr int kThreads = 320;                  // 10 warps
-    static constexpr int kNumBars = 2 * kSlots + 13;
+    static constexpr int kThreads = 384;                  // 3 warpgroups
+    // Registers: the launch gives every thread kLaunchRegs (the build checks
+    // ptxas reports exactly that); the softmax warpgroups then grow to
+    // kSoftmaxRegs and the producer/MMA warpgroup shrinks to kOtherRegs.
+    // 2 * 128 * kSoftmaxRegs + 128 * kOtherRegs must not exceed 384 * kLaunchRegs.
+    static constexpr int kLaunchRegs = 168;
+    static constexpr int kSoftmaxRegs = 192;
+    static constexpr int kOtherRegs = 120;
+    static_assert(2 * 128 * kSoftmaxRegs + 128 * kOtherRegs <= kThreads * kLaunchRegs,
+                  "register split exceeds the launch allocation");
+    static constexpr int kNumBars = 2 * kSlots + 15;   // FwdBars<kSlots>::kCount
     static constexpr int kSmemBytes = 1024 + (2 + kSlots) * kTileBytes + kNumBars * 8 + 16;
     static constexpr uint32_t kTmemCols = 512;
     static constexpr uint32_t kColS0 = 0, kColS1 = 128;
     static constexpr uint32_t kColO0 = 256, kColO1 = 256 + D;
 };
+
+#ifndef EATTN_POLY_EVERY
+#define EATTN_POLY_EVERY 0
+#endif
+// One exponent pair in every kPolyEvery goes to the FMA-pipe polynomial (0: none).
+constexpr int kPolyEvery = EATTN_POLY_EVERY;
+
+// Unit handled by this CTA in round r (snake order), or -1 past the end.
+__device__ __forceinline__ int fwd_unit_of_round(int r, int num_units) {
+    const int g = gridDim.x, i = blockIdx.x;
+    const long long u = (long long)r * g + ((r & 1) ? (g - 1 - i) : i);
+    return u < num_units ? (int)u : -1;
+}
+#define FWD_FOR_EACH_UNIT(u, p)                                                   \
+    for (int round_ = 0, u = 0; (long long)round_ * gridDim.x < (p).num_units; ++round_) \
+        if ((u = fwd_unit_of_round(round_, (p).num_units)) >= 0)
 
 struct FwdUnit {
     int bh, qb;
@@ -98,10 +140,24 @@ __device__ __forceinline__ FwdUnit fwd_unit(int u, const FwdParams& p) {
     return x;
 }
 
+// mbarrier addresses, all derived from one shared-memory base address so that
+// only a single register is live across the roles. Layout (8 bytes each):
+// kv_full[S], kv_empty[S], then 2 each of q_full, q_empty, s_full, p_lo, p_hi,
+// o_final, o_free, then drain.
+template <int S>
 struct FwdBars {
-    uint32_t kv_full, kv_empty;   // base addresses of the slot arrays (8 bytes apart)
-    uint32_t q_full, q_empty, s_full, p_ready, o_final, o_free;  // 2 each
-    uint32_t drain;
+    uint32_t base;
+    __device__ __forceinline__ uint32_t kv_full(uint32_t i) const { return base + 8 * i; }
+    __device__ __forceinline__ uint32_t kv_empty(uint32_t i) const { return base + 8 * (S + i); }
+    __device__ __forceinline__ uint32_t q_full(int t) const { return base + 8 * (2 * S + t); }
+    __device__ __forceinline__ uint32_t q_empty(int t) const { return base + 8 * (2 * S + 2 + t); }
+    __device__ __forceinline__ uint32_t s_full(int t) const { return base + 8 * (2 * S + 4 + t); }
+    __device__ __forceinline__ uint32_t p_lo(int t) const { return base + 8 * (2 * S + 6 + t); }
+    __device__ __forceinline__ uint32_t p_hi(int t) const { return base + 8 * (2 * S + 8 + t); }
+    __device__ __forceinline__ uint32_t o_final(int t) const { return base + 8 * (2 * S + 10 + t); }
+    __device__ __forceinline__ uint32_t o_free(int t) const { return base + 8 * (2 * S + 12 + t); }
+    __device__ __forceinline__ uint32_t drain() const { return base + 8 * (2 * S + 14); }
+    static constexpr int kCount = 2 * S + 15;
 };
 
 // Bounded wait executed by a whole warp; the outcome is made warp-uniform.
@@ -113,20 +169,20 @@ __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, volatil
 // ----------------------------------------------------------- TMA producer --
 template <int D, bool CAUSAL>
 __device__ void fwd_producer(const FwdParams& p, const CUtensorMap* tq, const CUtensorMap* tk,
-                             const CUtensorMap* tv, uint32_t sQ, uint32_t sKV, const FwdBars& b,
+                             const CUtensorMap* tv, uint32_t sQ, uint32_t sKV, const FwdBars<FwdTraits<D>::kSlots>& b,
                              volatile int* abort_flag) {
     using T = FwdTraits<D>;
     uint32_t kv_iter = 0;
     uint32_t q_issued[2] = {0, 0};
-    for (int u = blockIdx.x; u < p.num_units; u += gridDim.x) {
+    FWD_FOR_EACH_UNIT(u, p) {
         const FwdUnit x = fwd_unit<CAUSAL>(u, p);
         for (int t = 0; t < 2; ++t) {
             if (q_issued[t] > 0 &&
-                !mbar_wait(b.q_empty + 8 * t, (q_issued[t] - 1) & 1, abort_flag, &g_attn_status))
+                !mbar_wait(b.q_empty(t), (q_issued[t] - 1) & 1, abort_flag, &g_attn_status))
                 goto fail;
-            mbar_arrive_expect_tx(b.q_full + 8 * t, T::kTileBytes);
+            mbar_arrive_expect_tx(b.q_full(t), T::kTileBytes);
             for (int pn = 0; pn < T::kPanels; ++pn)
-                tma_load_3d(sQ + t * T::kTileBytes + pn * T::kPanelBytes, tq, b.q_full + 8 * t,
+                tma_load_3d(sQ + t * T::kTileBytes + pn * T::kPanelBytes, tq, b.q_full(t),
                             pn * 64, x.qb * 256 + t * 128, x.bh);
             ++q_issued[t];
         }
@@ -135,12 +191,12 @@ __device__ void fwd_producer(const FwdParams& p, const CUtensorMap* tq, const CU
                 const uint32_t slot = kv_iter % T::kSlots;
                 const uint32_t round = kv_iter / T::kSlots;
                 if (round > 0 &&
-                    !mbar_wait(b.kv_empty + 8 * slot, (round - 1) & 1, abort_flag, &g_attn_status))
+                    !mbar_wait(b.kv_empty(slot), (round - 1) & 1, abort_flag, &g_attn_status))
                     goto fail;
-                mbar_arrive_expect_tx(b.kv_full + 8 * slot, T::kTileBytes);
+                mbar_arrive_expect_tx(b.kv_full(slot), T::kTileBytes);
                 for (int pn = 0; pn < T::kPanels; ++pn)
                     tma_load_3d(sKV + slot * T::kTileBytes + pn * T::kPanelBytes,
-                                which ? tv : tk, b.kv_full + 8 * slot, pn * 64, j * 128, x.bh);
+                                which ? tv : tk, b.kv_full(slot), pn * 64, j * 128, x.bh);
                 ++kv_iter;
             }
         }
@@ -152,11 +208,11 @@ fail: {
     volatile int no_abort = 0;
     const uint32_t first = kv_iter > (uint32_t)T::kSlots ? kv_iter - T::kSlots : 0;
     for (uint32_t i = first; i < kv_iter; ++i)
-        mbar_wait(b.kv_full + 8 * (i % T::kSlots), (i / T::kSlots) & 1, &no_abort,
+        mbar_wait(b.kv_full(i % T::kSlots), (i / T::kSlots) & 1, &no_abort,
                   &g_attn_status);
     for (int t = 0; t < 2; ++t)
         if (q_issued[t] > 0)
-            mbar_wait(b.q_full + 8 * t, (q_issued[t] - 1) & 1, &no_abort, &g_attn_status);
+            mbar_wait(b.q_full(t), (q_issued[t] - 1) & 1, &no_abort, &g_attn_status);
 }
 }
 
@@ -175,11 +231,11 @@ __device__ __forceinline__ void fwd_issue_s(uint32_t tmem_s, uint32_t sQt, uint3
 
 template <int D>
 __device__ __forceinline__ void fwd_issue_pv(uint32_t tmem_o, uint32_t tmem_p, uint32_t sV,
-                                             bool accumulate) {
+                                             bool accumulate, int half) {
     using T = FwdTraits<D>;
     constexpr uint32_t idesc = idesc_bf16_f32(128, D, true);
 #pragma unroll
-    for (int kk = 0; kk < 128 / 16; ++kk) {
+    for (int kk = 4 * half; kk < 4 * half + 4; ++kk) {
         // P: 16 keys = 8 TMEM columns of bf16 pairs. V: 16 keys = 2 swizzle
         // atoms of 8 rows (2048 bytes); the two 64-column panels are kPanelBytes apart.
         mma_bf16_ts(tmem_o, tmem_p + kk * 8, sdesc_sw128(sV + kk * 2048, T::kPanelBytes, 1024),
@@ -189,20 +245,20 @@ __device__ __forceinline__ void fwd_issue_pv(uint32_t tmem_o, uint32_t tmem_p, u
 
 template <int D, bool CAUSAL>
 __device__ void fwd_mma(const FwdParams& p, uint32_t tbase, uint32_t sQ, uint32_t sKV,
-                        const FwdBars& b, volatile int* abort_flag) {
+                        const FwdBars<FwdTraits<D>::kSlots>& b, volatile int* abort_flag) {
     using T = FwdTraits<D>;
     const uint32_t colS[2] = {T::kColS0, T::kColS1};
     const uint32_t colO[2] = {T::kColO0, T::kColO1};
     uint32_t kv_iter = 0, q_use = 0;
     uint32_t o_use[2] = {0, 0}, p_phase[2] = {0, 0};
-    for (int u = blockIdx.x; u < p.num_units; u += gridDim.x) {
+    FWD_FOR_EACH_UNIT(u, p) {
         const FwdUnit x = fwd_unit<CAUSAL>(u, p);
-        if (!mbar_wait(b.q_full, q_use & 1, abort_flag, &g_attn_status)) goto done;
-        if (!mbar_wait(b.q_full + 8, q_use & 1, abort_flag, &g_attn_status)) goto done;
+        if (!mbar_wait(b.q_full(0), q_use & 1, abort_flag, &g_attn_status)) goto done;
+        if (!mbar_wait(b.q_full(1), q_use & 1, abort_flag, &g_attn_status)) goto done;
         tc_fence_after_sync();
         if (x.nmax > 0) {
             uint32_t kslot = kv_iter % T::kSlots;
-            if (!mbar_wait(b.kv_full + 8 * kslot, (kv_iter / T::kSlots) & 1, abort_flag,
+            if (!mbar_wait(b.kv_full(kslot), (kv_iter / T::kSlots) & 1, abort_flag,
                            &g_attn_status))
                 goto done;
             tc_fence_after_sync();
@@ -210,13 +266,13 @@ __device__ void fwd_mma(const FwdParams& p, uint32_t tbase, uint32_t sQ, uint32_
                 if (x.n[t] > 0) {
                     fwd_issue_s<D>(tbase + colS[t], sQ + t * T::kTileBytes,
                                    sKV + kslot * T::kTileBytes);
-                    mma_commit(b.s_full + 8 * t);
+                    mma_commit(b.s_full(t));
                 }
-            mma_commit(b.kv_empty + 8 * kslot);
+            mma_commit(b.kv_empty(kslot));
             ++kv_iter;
             for (int j = 0; j < x.nmax; ++j) {
                 const uint32_t vslot = kv_iter % T::kSlots;
-                if (!mbar_wait(b.kv_full + 8 * vslot, (kv_iter / T::kSlots) & 1, abort_flag,
+                if (!mbar_wait(b.kv_full(vslot), (kv_iter / T::kSlots) & 1, abort_flag,
                                &g_attn_status))
                     goto done;
                 tc_fence_after_sync();
@@ -226,38 +282,43 @@ __device__ void fwd_mma(const FwdParams& p, uint32_t tbase, uint32_t sQ, uint32_
                 const uint32_t kpar = (kv_iter / T::kSlots) & 1;
                 for (int t = 0; t < 2; ++t) {
                     if (j < x.n[t]) {
-                        if (!mbar_wait(b.p_ready + 8 * t, p_phase[t], abort_flag, &g_attn_status))
+                        if (!mbar_wait(b.p_lo(t), p_phase[t], abort_flag, &g_attn_status))
                             goto done;
-                        p_phase[t] ^= 1;
                         if (j == 0 && o_use[t] > 0 &&
-                            !mbar_wait(b.o_free + 8 * t, (o_use[t] - 1) & 1, abort_flag,
+                            !mbar_wait(b.o_free(t), (o_use[t] - 1) & 1, abort_flag,
                                        &g_attn_status))
                             goto done;
                         tc_fence_after_sync();
                         fwd_issue_pv<D>(tbase + colO[t], tbase + colS[t],
-                                        sKV + vslot * T::kTileBytes, j > 0);
-                        if (j == x.n[t] - 1) mma_commit(b.o_final + 8 * t);
+                                        sKV + vslot * T::kTileBytes, j > 0, 0);
+                        if (!mbar_wait(b.p_hi(t), p_phase[t], abort_flag, &g_attn_status))
+                            goto done;
+                        tc_fence_after_sync();
+                        fwd_issue_pv<D>(tbase + colO[t], tbase + colS[t],
+                                        sKV + vslot * T::kTileBytes, true, 1);
+                        p_phase[t] ^= 1;
+                        if (j == x.n[t] - 1) mma_commit(b.o_final(t));
                     }
                     if (t == 0 && has_next) {
-                        if (!mbar_wait(b.kv_full + 8 * kslot, kpar, abort_flag, &g_attn_status))
+                        if (!mbar_wait(b.kv_full(kslot), kpar, abort_flag, &g_attn_status))
                             goto done;
                         tc_fence_after_sync();
                     }
-                    if (t == 1) mma_commit(b.kv_empty + 8 * vslot);
+                    if (t == 1) mma_commit(b.kv_empty(vslot));
                     if (j + 1 < x.n[t]) {
                         fwd_issue_s<D>(tbase + colS[t], sQ + t * T::kTileBytes,
                                        sKV + kslot * T::kTileBytes);
-                        mma_commit(b.s_full + 8 * t);
+                        mma_commit(b.s_full(t));
                     }
                 }
                 if (has_next) {
-                    mma_commit(b.kv_empty + 8 * kslot);
+                    mma_commit(b.kv_empty(kslot));
                     ++kv_iter;
                 }
             }
         }
-        mma_commit(b.q_empty);
-        mma_commit(b.q_empty + 8);
+        mma_commit(b.q_empty(0));
+        mma_commit(b.q_empty(1));
         ++q_use;
         for (int t = 0; t < 2; ++t)
             if (x.n[t] > 0) ++o_use[t];
@@ -265,14 +326,14 @@ __device__ void fwd_mma(const FwdParams& p, uint32_t tbase, uint32_t sQ, uint32_
 done: {
     // Every MMA issued so far must finish before tensor memory is released.
     volatile int no_abort = 0;
-    mma_commit(b.drain);
-    mbar_wait(b.drain, 0, &no_abort, &g_attn_status);
+    mma_commit(b.drain());
+    mbar_wait(b.drain(), 0, &no_abort, &g_attn_status);
 }
 }
 
 // --------------------------------------------------------------- softmax --
 template <int D, bool CAUSAL>
-__device__ void fwd_softmax(const FwdParams& p, uint32_t tbase, const FwdBars& b, int warp,
+__device__ void fwd_softmax(const FwdParams& p, uint32_t tbase, const FwdBars<FwdTraits<D>::kSlots>& b, int warp,
                             int lane, volatile int* abort_flag) {
     using T = FwdTraits<D>;
     const int t = warp >> 2;                 // which Q tile
@@ -281,18 +342,20 @@ __device__ void fwd_softmax(const FwdParams& p, uint32_t tbase, const FwdBars& b
     const uint32_t lane_off = uint32_t(quarter * 32) << 16;
     const uint32_t tS = tbase + lane_off + (t ? T::kColS1 : T::kColS0);
     const uint32_t tO = tbase + lane_off + (t ? T::kColO1 : T::kColO0);
-    const uint32_t bar_s = b.s_full + 8 * t, bar_p = b.p_ready + 8 * t;
-    const uint32_t bar_of = b.o_final + 8 * t, bar_ofree = b.o_free + 8 * t;
+    const uint32_t bar_s = b.s_full(t);
+    const uint32_t bar_plo = b.p_lo(t), bar_phi = b.p_hi(t);
+    const uint32_t bar_of = b.o_final(t), bar_ofree = b.o_free(t);
     const float c2 = p.scale_log2;
     uint32_t s_phase = 0, o_use = 0;
 
-    for (int u = blockIdx.x; u < p.num_units; u += gridDim.x) {
+    FWD_FOR_EACH_UNIT(u, p) {
         const FwdUnit x = fwd_unit<CAUSAL>(u, p);
         const int n = x.n[t];
-        const long long qrow = (long long)x.qb * 256 + t * 128 + r;
+        // sequence lengths are at most 2^30, so row indices and limits fit in int
+        const int qrow = x.qb * 256 + t * 128 + r;
         const bool row_valid = qrow < p.Nq;
-        long long kv_lim = p.Nkv;   // keys [0, kv_lim) are visible to this row
-        if (CAUSAL) kv_lim = min(kv_lim, qrow + ((long long)p.Nkv - p.Nq) + 1);
+        int kv_lim = p.Nkv;         // keys [0, kv_lim) are visible to this row
+        if (CAUSAL) kv_lim = min(kv_lim, qrow + (p.Nkv - p.Nq) + 1);
         float m_ref = -INFINITY;    // reference max, log2 units (scaled)
         float l = 0.f;              // running sum of 2^(s*c2 - m_ref)
 
@@ -303,62 +366,86 @@ __device__ void fwd_softmax(const FwdParams& p, uint32_t tbase, const FwdBars& b
             uint32_t sr[128];
             tmem_ld128(tS, sr);
             tmem_wait_ld128(sr);
-            const long long lim = kv_lim - (long long)j * 128;
-            if (lim < 128) {
+            {
+                // columns c >= lim of this tile are masked (-inf) for this row
+                const int lim = max(-1, min(128, kv_lim - j * 128));
+                if (lim < 128) {
 #pragma unroll
-                for (int c = 0; c < 128; ++c)
-                    if (c >= lim) sr[c] = __float_as_uint(-INFINITY);
+                    for (int c = 0; c < 128; ++c)
+                        if (c >= lim) sr[c] = __float_as_uint(-INFINITY);
+                }
             }
-            float mx0 = __uint_as_float(sr[0]), mx1 = __uint_as_float(sr[1]);
-            float mx2 = __uint_as_float(sr[2]), mx3 = __uint_as_float(sr[3]);
+            float mx0 = -INFINITY, mx1 = -INFINITY, mx2 = -INFINITY, mx3 = -INFINITY;
 #pragma unroll
-            for (int c = 4; c < 128; c += 4) {
-                mx0 = fmaxf(mx0, __uint_as_float(sr[c]));
-                mx1 = fmaxf(mx1, __uint_as_float(sr[c + 1]));
-                mx2 = fmaxf(mx2, __uint_as_float(sr[c + 2]));
-                mx3 = fmaxf(mx3, __uint_as_float(sr[c + 3]));
+            for (int c = 0; c < 128; c += 8) {
+                mx0 = fmax3(mx0, __uint_as_float(sr[c]), __uint_as_float(sr[c + 1]));
+                mx1 = fmax3(mx1, __uint_as_float(sr[c + 2]), __uint_as_float(sr[c + 3]));
+                mx2 = fmax3(mx2, __uint_as_float(sr[c + 4]), __uint_as_float(sr[c + 5]));
+                mx3 = fmax3(mx3, __uint_as_float(sr[c + 6]), __uint_as_float(sr[c + 7]));
             }
-            const float mxs = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * c2;
+            const float mxs = fmax3(mx0, mx1, fmaxf(mx2, mx3)) * c2;
             const bool need = mxs > m_ref + 8.0f;
             const bool any_need = __any_sync(0xffffffffu, need);
             const float m_new = need ? mxs : m_ref;
             const float alpha = need ? fast_exp2(m_ref - m_new) : 1.0f;
             m_ref = m_new;
             const float base = (m_ref == -INFINITY) ? 0.f : m_ref;
-            uint32_t pk[64];
-            float l0 = 0.f, l1 = 0.f;
+            const f32x2_t c2x2 = f2_pack(c2, c2);
+            const f32x2_t nbx2 = f2_pack(-base, -base);
+            f32x2_t lsum_a = f2_pack(0.f, 0.f), lsum_b = f2_pack(0.f, 0.f);
 #pragma unroll
-            for (int i = 0; i < 64; ++i) {
-                const float e0 = fast_exp2(fmaf(__uint_as_float(sr[2 * i]), c2, -base));
-                const float e1 = fast_exp2(fmaf(__uint_as_float(sr[2 * i + 1]), c2, -base));
-                l0 += e0;
-                l1 += e1;
-                pk[i] = pack_bf16x2(e0, e1);
-            }
-            l = l * alpha + (l0 + l1);
-            tmem_st64(tS, pk);
-            if (any_need && j > 0) {
-                // Rescale O_t by alpha (1 for rows whose max did not move).
-                // O_t is stable here: the commit that signalled S_t(j) also
-                // covers the earlier P_t(j-1) V product, and P_t(j) V is not
-                // issued before this group arrives on p_ready.
+            for (int h = 0; h < 2; ++h) {
+                uint32_t pk[32];
 #pragma unroll
-                for (int c = 0; c < D; c += 32) {
-                    uint32_t orr[32];
-                    tmem_ld32(tO + c, orr);
-                    tmem_wait_ld(orr);
-#pragma unroll
-                    for (int i = 0; i < 32; ++i)
-                        orr[i] = __float_as_uint(__uint_as_float(orr[i]) * alpha);
-                    tmem_st32(tO + c, orr);
+                for (int i = 0; i < 32; ++i) {
+                    const int c = 64 * h + 2 * i;
+                    const f32x2_t xv = f2_fma(
+                        f2_pack(__uint_as_float(sr[c]), __uint_as_float(sr[c + 1])), c2x2, nbx2);
+                    float e0, e1;
+                    if (kPolyEvery > 0 && (i % (kPolyEvery > 0 ? kPolyEvery : 1)) == kPolyEvery - 1) {
+                        exp2_poly_pair(xv, e0, e1);
+                    } else {
+                        float x0, x1;
+                        f2_unpack(xv, x0, x1);
+                        e0 = fast_exp2(x0);
+                        e1 = fast_exp2(x1);
+                    }
+                    if (i & 1)
+                        lsum_b = f2_add(lsum_b, f2_pack(e0, e1));
+                    else
+                        lsum_a = f2_add(lsum_a, f2_pack(e0, e1));
+                    pk[i] = pack_bf16x2(e0, e1);
                 }
+                if (h == 0 && any_need && j > 0) {
+                    // Rescale O_t by alpha (1 for rows whose max did not move)
+                    // before any of P_t(j) V is released. O_t is stable here: the
+                    // commit that signalled S_t(j) also covers P_t(j-1) V.
+#pragma unroll
+                    for (int c = 0; c < D; c += 32) {
+                        uint32_t orr[32];
+                        tmem_ld32(tO + c, orr);
+                        tmem_wait_ld(orr);
+#pragma unroll
+                        for (int q = 0; q < 32; ++q)
+                            orr[q] = __float_as_uint(__uint_as_float(orr[q]) * alpha);
+                        tmem_st32(tO + c, orr);
+                    }
+                }
+                tmem_st32(tS + 32 * h, pk);
+                tmem_wait_st();
+                tc_fence_before_sync();
+                mbar_arrive(h == 0 ? bar_plo : bar_phi);
             }
-            tmem_wait_st();
-            tc_fence_before_sync();
-            mbar_arrive(bar_p);
+            float la0, la1, lb0, lb1;
+            f2_unpack(lsum_a, la0, la1);
+            f2_unpack(lsum_b, lb0, lb1);
+            l = l * alpha + ((la0 + la1) + (lb0 + lb1));
         }
 
         uint16_t* orow = p.o + ((size_t)x.bh * p.Nq + (size_t)(row_valid ? qrow : 0)) * D;
+        // A row that sees no key at all (causal with Nq > Nkv) is O = 0, LSE = -inf by
+        // definition; its polynomial exponentials of -inf scores are tiny, not zero.
+        if (kv_lim <= 0) l = 0.f;
         if (n > 0) {
             if (!warp_wait(bar_of, o_use & 1, abort_flag)) return;
             tc_fence_after_sync();
@@ -396,7 +483,7 @@ __device__ void fwd_softmax(const FwdParams& p, uint32_t tbase, const FwdBars& b
 
 // ---------------------------------------------------------------- kernel --
 template <int D, bool CAUSAL>
-__global__ void __launch_bounds__(320, 1)
+__global__ void __launch_bounds__(384, 1)
     attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
                           const __grid_constant__ CUtensorMap tm_k,
                           const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
@@ -408,17 +495,9 @@ __global__ void __launch_bounds__(320, 1)
     const uint32_t sKV = sQ + 2 * T::kTileBytes;
     uint8_t* bar_ptr = smem + (2 + T::kSlots) * T::kTileBytes;
     const uint32_t bar0 = smem_addr(bar_ptr);
-    FwdBars b;
-    b.kv_full = bar0;
-    b.kv_empty = bar0 + 8 * T::kSlots;
-    b.q_full = bar0 + 16 * T::kSlots;
-    b.q_empty = b.q_full + 16;
-    b.s_full = b.q_empty + 16;
-    b.p_ready = b.s_full + 16;
-    b.o_final = b.p_ready + 16;
-    b.o_free = b.o_final + 16;
-    b.drain = b.o_free + 16;
-    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bar_ptr + 8 * T::kNumBars);
+    FwdBars<T::kSlots> b;
+    b.base = bar0;
+    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bar_ptr + 8 * FwdBars<T::kSlots>::kCount);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
 
     const int warp = threadIdx.x >> 5;
@@ -426,18 +505,19 @@ __global__ void __launch_bounds__(320, 1)
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < T::kSlots; ++i) {
-            mbar_init(b.kv_full + 8 * i, 1);
-            mbar_init(b.kv_empty + 8 * i, 1);
+            mbar_init(b.kv_full(i), 1);
+            mbar_init(b.kv_empty(i), 1);
         }
         for (int t = 0; t < 2; ++t) {
-            mbar_init(b.q_full + 8 * t, 1);
-            mbar_init(b.q_empty + 8 * t, 1);
-            mbar_init(b.s_full + 8 * t, 1);
-            mbar_init(b.p_ready + 8 * t, 128);
-            mbar_init(b.o_final + 8 * t, 1);
-            mbar_init(b.o_free + 8 * t, 128);
+            mbar_init(b.q_full(t), 1);
+            mbar_init(b.q_empty(t), 1);
+            mbar_init(b.s_full(t), 1);
+            mbar_init(b.p_lo(t), 128);
+            mbar_init(b.p_hi(t), 128);
+            mbar_init(b.o_final(t), 1);
+            mbar_init(b.o_free(t), 128);
         }
-        mbar_init(b.drain, 1);
+        mbar_init(b.drain(), 1);
         *abort_flag = 0;
         fence_mbar_init();
     }
@@ -456,11 +536,14 @@ __global__ void __launch_bounds__(320, 1)
     const uint32_t tbase = *tmem_holder;
 
     if (warp < 8) {
+        regs_increase<T::kSoftmaxRegs>();
         fwd_softmax<D, CAUSAL>(p, tbase, b, warp, lane, abort_flag);
-    } else if (warp == 8) {
-        if (lane == 0) fwd_producer<D, CAUSAL>(p, &tm_q, &tm_k, &tm_v, sQ, sKV, b, abort_flag);
     } else {
-        if (lane == 0) fwd_mma<D, CAUSAL>(p, tbase, sQ, sKV, b, abort_flag);
+        regs_decrease<T::kOtherRegs>();
+        if (warp == 8 && lane == 0)
+            fwd_producer<D, CAUSAL>(p, &tm_q, &tm_k, &tm_v, sQ, sKV, b, abort_flag);
+        else if (warp == 9 && lane == 0)
+            fwd_mma<D, CAUSAL>(p, tbase, sQ, sKV, b, abort_flag);
     }
 
     tc_fence_before_sync();

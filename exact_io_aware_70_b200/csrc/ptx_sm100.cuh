@@ -65,7 +65,7 @@ __device__ __forceinline__ bool mbar_test(uint32_t bar, uint32_t parity) {
 
 // Bounded wait for the phase of `bar` with the given parity to complete.
 // `abort_flag` is the CTA's shared abort word. Returns false on give-up.
-__device__ __noinline__ bool mbar_wait_slow(uint32_t bar, uint32_t parity,
+__device__ __forceinline__ bool mbar_wait_slow(uint32_t bar, uint32_t parity,
                                             volatile int* abort_flag, unsigned* status) {
     const unsigned long long t0 = global_timer_ns();
     for (unsigned polls = 0; polls < kWaitMaxPolls; ++polls) {
@@ -117,6 +117,16 @@ __device__ __forceinline__ void tmem_relinquish() {
 __device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
                  : "memory");
+}
+
+// Per-warpgroup register budget (executed by all warps of a warpgroup).
+template <int N>
+__device__ __forceinline__ void regs_increase() {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <int N>
+__device__ __forceinline__ void regs_decrease() {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
 }
 
 __device__ __forceinline__ void tc_fence_before_sync() {
@@ -231,6 +241,67 @@ __device__ __forceinline__ void tmem_wait_st() {
 }
 
 // ------------------------------------------------------------ arithmetic --
+// Packed pair of fp32 values in one 64-bit register (sm_100 f32x2 instructions).
+typedef unsigned long long f32x2_t;
+
+__device__ __forceinline__ f32x2_t f2_pack(float lo, float hi) {
+    f32x2_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+    return r;
+}
+__device__ __forceinline__ void f2_unpack(f32x2_t v, float& lo, float& hi) {
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ f32x2_t f2_fma(f32x2_t a, f32x2_t b, f32x2_t c) {
+    f32x2_t d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    return d;
+}
+__device__ __forceinline__ f32x2_t f2_add(f32x2_t a, f32x2_t b) {
+    f32x2_t d;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+
+// max of three floats in one instruction (sm_100)
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+    float d;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+    return d;
+}
+
+// 2^x for a pair of finite x <= 126 on the FMA pipe instead of the MUFU unit.
+// Range reduction x = n + f with n = round-to-nearest(x) (obtained by adding
+// and subtracting 1.5 * 2^23 in round-to-nearest-even), f in [-1/2, 1/2];
+// 2^f from a degree-3 polynomial whose coefficients were fitted for this
+// library by a Remez exchange minimising the relative error on [-1/2, 1/2]
+// (max relative error 7.5e-5, well below the 2^-9 rounding of a bf16 P);
+// then 2^n is applied by adding n to the exponent field. Inputs below -125
+// are clamped there (result about 2^-125, negligible next to the row sum,
+// which is at least 1). Callers only use this on tiles without masked (-inf)
+// scores.
+constexpr float kExp2C0 = 0.9999280571937561f;
+constexpr float kExp2C1 = 0.6932609677314758f;
+constexpr float kExp2C2 = 0.2426111251115799f;
+constexpr float kExp2C3 = 0.0551716685295105f;
+constexpr float kRoundMagic = 12582912.0f;   // 1.5 * 2^23
+
+__device__ __forceinline__ void exp2_poly_pair(f32x2_t x, float& y0, float& y1) {
+    float x0, x1;
+    f2_unpack(x, x0, x1);
+    x = f2_pack(fmaxf(x0, -125.0f), fmaxf(x1, -125.0f));
+    const f32x2_t t = f2_add(x, f2_pack(kRoundMagic, kRoundMagic));       // n in the low bits
+    const f32x2_t n = f2_add(t, f2_pack(-kRoundMagic, -kRoundMagic));     // n as a float
+    const f32x2_t f = f2_fma(n, f2_pack(-1.0f, -1.0f), x);               // x - n
+    f32x2_t p = f2_fma(f2_pack(kExp2C3, kExp2C3), f, f2_pack(kExp2C2, kExp2C2));
+    p = f2_fma(p, f, f2_pack(kExp2C1, kExp2C1));
+    p = f2_fma(p, f, f2_pack(kExp2C0, kExp2C0));
+    float p0, p1, t0, t1;
+    f2_unpack(p, p0, p1);
+    f2_unpack(t, t0, t1);
+    y0 = __uint_as_float(__float_as_uint(p0) + (__float_as_uint(t0) << 23));
+    y1 = __uint_as_float(__float_as_uint(p1) + (__float_as_uint(t1) << 23));
+}
 __device__ __forceinline__ float fast_exp2(float x) {
     float y;
     asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));

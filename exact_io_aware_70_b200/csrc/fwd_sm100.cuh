@@ -18,10 +18,14 @@
 //     to the CTAs in alternating direction each round (CTA i takes unit
 //     r*G + i in even rounds, r*G + G-1-i in odd rounds), which balances the
 //     causal triangle across the 148 SMs about as well as longest-first greedy.
-//   * Warp 8 (one elected lane) is the TMA producer: Q tiles once per unit,
+//   * Warp 8 is the TMA producer (lane 0 issues): Q tiles once per unit,
 //     then K_j and V_j tiles into a ring of shared-memory slots, 128-byte
 //     swizzled, completion counted on mbarriers.
-//   * Warp 9 (one elected lane) issues every tcgen05.mma: S_t = Q_t K_j^T into
+//   * Warp 9 issues every tcgen05.mma from lane 0, with shared-memory
+//     descriptors precomputed per tile and advanced by constant offsets. A
+//     tcgen05.mma costs the issuing thread about 48 cycles (measured), close
+//     to the 64 cycles one 128x128x16 MMA keeps the tensor core busy, so this
+//     thread's loop is kept as short as possible.: S_t = Q_t K_j^T into
 //     tensor memory (fp32, 128x128), and O_t += P_t V_j with P_t read straight
 //     from tensor memory (bf16, aliased over S_t's first 64 columns).
 //   * 384 threads = 3 warpgroups; warps 10-11 only complete the third
@@ -70,6 +74,10 @@ struct FwdParams {
     float scale_log2;   // scale * log2(e)
 };
 
+#ifndef EATTN_KV_SLOTS_D128
+#define EATTN_KV_SLOTS_D128 4
+#endif
+
 template <int D>
 struct FwdTraits {
     static_assert(D == 64 || D == 128, "head dim 64 or 128");
@@ -77,7 +85,8 @@ struct FwdTraits {
     static constexpr int kPanelBytes = 128 * 64 * 2;      // 128 rows x 64 bf16 (one swizzle panel)
     static constexpr int kPanels = D / 64;
     static constexpr int kTileBytes = kPanels * kPanelBytes;
-    static constexpr int kSlots = (D == 128) ? 4 : 8;     // K/V ring depth (tiles)
+    static constexpr int kSlots = (D == 128) ? EATTN_KV_SLOTS_D128 : 8;   // K/V ring depth (tiles)
+    static_assert(kSlots >= 2, "the ring holds K_j and V_j at once");
     static constexpr int kThreads = 384;                  // 3 warpgroups
     // Registers: the launch gives every thread kLaunchRegs (the build checks
     // ptxas reports exactly that); the softmax warpgroups then grow to
@@ -90,6 +99,7 @@ struct FwdTraits {
                   "register split exceeds the launch allocation");
     static constexpr int kNumBars = 2 * kSlots + 15;   // FwdBars<kSlots>::kCount
     static constexpr int kSmemBytes = 1024 + (2 + kSlots) * kTileBytes + kNumBars * 8 + 16;
+    static_assert(kSmemBytes <= 232448, "shared memory per CTA");
     static constexpr uint32_t kTmemCols = 512;
     static constexpr uint32_t kColS0 = 0, kColS1 = 128;
     static constexpr uint32_t kColO0 = 256, kColO1 = 256 + D;
@@ -166,10 +176,26 @@ __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, volatil
     return __all_sync(0xffffffffu, ok);
 }
 
+// The producer and MMA roles run either on one lane (EATTN_WARP_ISSUE 0: the
+// other 31 lanes go straight to the final barrier) or on the whole warp with
+// converged control flow and only lane 0 issuing (EATTN_WARP_ISSUE 1).
+#ifndef EATTN_WARP_ISSUE
+#define EATTN_WARP_ISSUE 0
+#endif
+__device__ __forceinline__ bool role_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag) {
+#if EATTN_WARP_ISSUE
+    return warp_wait(bar, parity, abort_flag);
+#else
+    return mbar_wait(bar, parity, abort_flag, &g_attn_status);
+#endif
+}
+
 // ----------------------------------------------------------- TMA producer --
+// Run by the whole producer warp with converged control flow; lane 0 issues.
 template <int D, bool CAUSAL>
 __device__ void fwd_producer(const FwdParams& p, const CUtensorMap* tq, const CUtensorMap* tk,
-                             const CUtensorMap* tv, uint32_t sQ, uint32_t sKV, const FwdBars<FwdTraits<D>::kSlots>& b,
+                             const CUtensorMap* tv, uint32_t sQ, uint32_t sKV,
+                             const FwdBars<FwdTraits<D>::kSlots>& b, uint32_t leader,
                              volatile int* abort_flag) {
     using T = FwdTraits<D>;
     uint32_t kv_iter = 0;
@@ -177,26 +203,27 @@ __device__ void fwd_producer(const FwdParams& p, const CUtensorMap* tq, const CU
     FWD_FOR_EACH_UNIT(u, p) {
         const FwdUnit x = fwd_unit<CAUSAL>(u, p);
         for (int t = 0; t < 2; ++t) {
-            if (q_issued[t] > 0 &&
-                !mbar_wait(b.q_empty(t), (q_issued[t] - 1) & 1, abort_flag, &g_attn_status))
+            if (q_issued[t] > 0 && !role_wait(b.q_empty(t), (q_issued[t] - 1) & 1, abort_flag))
                 goto fail;
-            mbar_arrive_expect_tx(b.q_full(t), T::kTileBytes);
+            mbar_arrive_expect_tx_w(b.q_full(t), T::kTileBytes, leader);
+#pragma unroll
             for (int pn = 0; pn < T::kPanels; ++pn)
-                tma_load_3d(sQ + t * T::kTileBytes + pn * T::kPanelBytes, tq, b.q_full(t),
-                            pn * 64, x.qb * 256 + t * 128, x.bh);
+                tma_load_3d_w(sQ + t * T::kTileBytes + pn * T::kPanelBytes, tq, b.q_full(t),
+                              pn * 64, x.qb * 256 + t * 128, x.bh, leader);
             ++q_issued[t];
         }
         for (int j = 0; j < x.nmax; ++j) {
+#pragma unroll
             for (int which = 0; which < 2; ++which) {   // K_j, then V_j
                 const uint32_t slot = kv_iter % T::kSlots;
                 const uint32_t round = kv_iter / T::kSlots;
-                if (round > 0 &&
-                    !mbar_wait(b.kv_empty(slot), (round - 1) & 1, abort_flag, &g_attn_status))
+                if (round > 0 && !role_wait(b.kv_empty(slot), (round - 1) & 1, abort_flag))
                     goto fail;
-                mbar_arrive_expect_tx(b.kv_full(slot), T::kTileBytes);
+                mbar_arrive_expect_tx_w(b.kv_full(slot), T::kTileBytes, leader);
+#pragma unroll
                 for (int pn = 0; pn < T::kPanels; ++pn)
-                    tma_load_3d(sKV + slot * T::kTileBytes + pn * T::kPanelBytes,
-                                which ? tv : tk, b.kv_full(slot), pn * 64, j * 128, x.bh);
+                    tma_load_3d_w(sKV + slot * T::kTileBytes + pn * T::kPanelBytes,
+                                  which ? tv : tk, b.kv_full(slot), pn * 64, j * 128, x.bh, leader);
                 ++kv_iter;
             }
         }
@@ -208,8 +235,7 @@ fail: {
     volatile int no_abort = 0;
     const uint32_t first = kv_iter > (uint32_t)T::kSlots ? kv_iter - T::kSlots : 0;
     for (uint32_t i = first; i < kv_iter; ++i)
-        mbar_wait(b.kv_full(i % T::kSlots), (i / T::kSlots) & 1, &no_abort,
-                  &g_attn_status);
+        mbar_wait(b.kv_full(i % T::kSlots), (i / T::kSlots) & 1, &no_abort, &g_attn_status);
     for (int t = 0; t < 2; ++t)
         if (q_issued[t] > 0)
             mbar_wait(b.q_full(t), (q_issued[t] - 1) & 1, &no_abort, &g_attn_status);
@@ -217,63 +243,69 @@ fail: {
 }
 
 // ------------------------------------------------------------ MMA issuer --
+// Descriptor bases are computed once; an operand at byte offset `off` from a
+// base is the base plus off >> 4 (the start-address field never overflows:
+// shared memory addresses are below 2^18).
 template <int D>
-__device__ __forceinline__ void fwd_issue_s(uint32_t tmem_s, uint32_t sQt, uint32_t sK) {
+__device__ __forceinline__ void fwd_issue_s(uint32_t tmem_s, uint64_t dq, uint64_t dk,
+                                            uint32_t leader) {
     using T = FwdTraits<D>;
     constexpr uint32_t idesc = idesc_bf16_f32(128, 128, false);
 #pragma unroll
     for (int kk = 0; kk < D / 16; ++kk) {
-        const uint32_t off = (kk / 4) * T::kPanelBytes + (kk % 4) * 32;
-        mma_bf16_ss(tmem_s, sdesc_sw128(sQt + off, 16, 1024), sdesc_sw128(sK + off, 16, 1024),
-                    idesc, kk > 0 ? 1u : 0u);
+        const uint64_t off = ((kk / 4) * T::kPanelBytes + (kk % 4) * 32) >> 4;
+        mma_bf16_ss_w(tmem_s, dq + off, dk + off, idesc, kk > 0 ? 1u : 0u, leader);
     }
 }
 
 template <int D>
-__device__ __forceinline__ void fwd_issue_pv(uint32_t tmem_o, uint32_t tmem_p, uint32_t sV,
-                                             bool accumulate, int half) {
-    using T = FwdTraits<D>;
+__device__ __forceinline__ void fwd_issue_pv(uint32_t tmem_o, uint32_t tmem_p, uint64_t dv,
+                                             bool accumulate, int half, uint32_t leader) {
     constexpr uint32_t idesc = idesc_bf16_f32(128, D, true);
 #pragma unroll
     for (int kk = 4 * half; kk < 4 * half + 4; ++kk) {
         // P: 16 keys = 8 TMEM columns of bf16 pairs. V: 16 keys = 2 swizzle
-        // atoms of 8 rows (2048 bytes); the two 64-column panels are kPanelBytes apart.
-        mma_bf16_ts(tmem_o, tmem_p + kk * 8, sdesc_sw128(sV + kk * 2048, T::kPanelBytes, 1024),
-                    idesc, (accumulate || kk > 0) ? 1u : 0u);
+        // atoms of 8 rows (2048 bytes); the 64-column panels are kPanelBytes
+        // apart (the descriptor's leading-dimension offset).
+        mma_bf16_ts_w(tmem_o, tmem_p + kk * 8, dv + ((kk * 2048) >> 4), idesc,
+                      (accumulate || kk > 0) ? 1u : 0u, leader);
     }
 }
 
+// Run by the whole MMA warp with converged control flow; lane 0 issues.
 template <int D, bool CAUSAL>
 __device__ void fwd_mma(const FwdParams& p, uint32_t tbase, uint32_t sQ, uint32_t sKV,
-                        const FwdBars<FwdTraits<D>::kSlots>& b, volatile int* abort_flag) {
+                        const FwdBars<FwdTraits<D>::kSlots>& b, uint32_t leader,
+                        volatile int* abort_flag) {
     using T = FwdTraits<D>;
+    constexpr uint64_t kTileStep = T::kTileBytes >> 4;
+    const uint64_t dq0 = sdesc_sw128(sQ, 16, 1024);
+    const uint64_t dk0 = sdesc_sw128(sKV, 16, 1024);                  // K-major K tile
+    const uint64_t dv0 = sdesc_sw128(sKV, T::kPanelBytes, 1024);      // MN-major V tile
     const uint32_t colS[2] = {T::kColS0, T::kColS1};
     const uint32_t colO[2] = {T::kColO0, T::kColO1};
     uint32_t kv_iter = 0, q_use = 0;
     uint32_t o_use[2] = {0, 0}, p_phase[2] = {0, 0};
     FWD_FOR_EACH_UNIT(u, p) {
         const FwdUnit x = fwd_unit<CAUSAL>(u, p);
-        if (!mbar_wait(b.q_full(0), q_use & 1, abort_flag, &g_attn_status)) goto done;
-        if (!mbar_wait(b.q_full(1), q_use & 1, abort_flag, &g_attn_status)) goto done;
+        if (!role_wait(b.q_full(0), q_use & 1, abort_flag)) goto done;
+        if (!role_wait(b.q_full(1), q_use & 1, abort_flag)) goto done;
         tc_fence_after_sync();
         if (x.nmax > 0) {
             uint32_t kslot = kv_iter % T::kSlots;
-            if (!mbar_wait(b.kv_full(kslot), (kv_iter / T::kSlots) & 1, abort_flag,
-                           &g_attn_status))
-                goto done;
+            if (!role_wait(b.kv_full(kslot), (kv_iter / T::kSlots) & 1, abort_flag)) goto done;
             tc_fence_after_sync();
             for (int t = 0; t < 2; ++t)
                 if (x.n[t] > 0) {
-                    fwd_issue_s<D>(tbase + colS[t], sQ + t * T::kTileBytes,
-                                   sKV + kslot * T::kTileBytes);
-                    mma_commit(b.s_full(t));
+                    fwd_issue_s<D>(tbase + colS[t], dq0 + t * kTileStep, dk0 + kslot * kTileStep,
+                                   leader);
+                    mma_commit_w(b.s_full(t), leader);
                 }
-            mma_commit(b.kv_empty(kslot));
+            mma_commit_w(b.kv_empty(kslot), leader);
             ++kv_iter;
             for (int j = 0; j < x.nmax; ++j) {
                 const uint32_t vslot = kv_iter % T::kSlots;
-                if (!mbar_wait(b.kv_full(vslot), (kv_iter / T::kSlots) & 1, abort_flag,
-                               &g_attn_status))
+                if (!role_wait(b.kv_full(vslot), (kv_iter / T::kSlots) & 1, abort_flag))
                     goto done;
                 tc_fence_after_sync();
                 ++kv_iter;
@@ -282,43 +314,39 @@ __device__ void fwd_mma(const FwdParams& p, uint32_t tbase, uint32_t sQ, uint32_
                 const uint32_t kpar = (kv_iter / T::kSlots) & 1;
                 for (int t = 0; t < 2; ++t) {
                     if (j < x.n[t]) {
-                        if (!mbar_wait(b.p_lo(t), p_phase[t], abort_flag, &g_attn_status))
-                            goto done;
+                        if (!role_wait(b.p_lo(t), p_phase[t], abort_flag)) goto done;
                         if (j == 0 && o_use[t] > 0 &&
-                            !mbar_wait(b.o_free(t), (o_use[t] - 1) & 1, abort_flag,
-                                       &g_attn_status))
+                            !role_wait(b.o_free(t), (o_use[t] - 1) & 1, abort_flag))
                             goto done;
                         tc_fence_after_sync();
-                        fwd_issue_pv<D>(tbase + colO[t], tbase + colS[t],
-                                        sKV + vslot * T::kTileBytes, j > 0, 0);
-                        if (!mbar_wait(b.p_hi(t), p_phase[t], abort_flag, &g_attn_status))
-                            goto done;
+                        fwd_issue_pv<D>(tbase + colO[t], tbase + colS[t], dv0 + vslot * kTileStep,
+                                        j > 0, 0, leader);
+                        if (!role_wait(b.p_hi(t), p_phase[t], abort_flag)) goto done;
                         tc_fence_after_sync();
-                        fwd_issue_pv<D>(tbase + colO[t], tbase + colS[t],
-                                        sKV + vslot * T::kTileBytes, true, 1);
+                        fwd_issue_pv<D>(tbase + colO[t], tbase + colS[t], dv0 + vslot * kTileStep,
+                                        true, 1, leader);
                         p_phase[t] ^= 1;
-                        if (j == x.n[t] - 1) mma_commit(b.o_final(t));
+                        if (j == x.n[t] - 1) mma_commit_w(b.o_final(t), leader);
                     }
                     if (t == 0 && has_next) {
-                        if (!mbar_wait(b.kv_full(kslot), kpar, abort_flag, &g_attn_status))
-                            goto done;
+                        if (!role_wait(b.kv_full(kslot), kpar, abort_flag)) goto done;
                         tc_fence_after_sync();
                     }
-                    if (t == 1) mma_commit(b.kv_empty(vslot));
+                    if (t == 1) mma_commit_w(b.kv_empty(vslot), leader);
                     if (j + 1 < x.n[t]) {
-                        fwd_issue_s<D>(tbase + colS[t], sQ + t * T::kTileBytes,
-                                       sKV + kslot * T::kTileBytes);
-                        mma_commit(b.s_full(t));
+                        fwd_issue_s<D>(tbase + colS[t], dq0 + t * kTileStep,
+                                       dk0 + kslot * kTileStep, leader);
+                        mma_commit_w(b.s_full(t), leader);
                     }
                 }
                 if (has_next) {
-                    mma_commit(b.kv_empty(kslot));
+                    mma_commit_w(b.kv_empty(kslot), leader);
                     ++kv_iter;
                 }
             }
         }
-        mma_commit(b.q_empty(0));
-        mma_commit(b.q_empty(1));
+        mma_commit_w(b.q_empty(0), leader);
+        mma_commit_w(b.q_empty(1), leader);
         ++q_use;
         for (int t = 0; t < 2; ++t)
             if (x.n[t] > 0) ++o_use[t];
@@ -326,7 +354,7 @@ __device__ void fwd_mma(const FwdParams& p, uint32_t tbase, uint32_t sQ, uint32_
 done: {
     // Every MMA issued so far must finish before tensor memory is released.
     volatile int no_abort = 0;
-    mma_commit(b.drain());
+    mma_commit_w(b.drain(), leader);
     mbar_wait(b.drain(), 0, &no_abort, &g_attn_status);
 }
 }
@@ -540,10 +568,11 @@ __global__ void __launch_bounds__(384, 1)
         fwd_softmax<D, CAUSAL>(p, tbase, b, warp, lane, abort_flag);
     } else {
         regs_decrease<T::kOtherRegs>();
-        if (warp == 8 && lane == 0)
-            fwd_producer<D, CAUSAL>(p, &tm_q, &tm_k, &tm_v, sQ, sKV, b, abort_flag);
-        else if (warp == 9 && lane == 0)
-            fwd_mma<D, CAUSAL>(p, tbase, sQ, sKV, b, abort_flag);
+        const bool issuer_thread = EATTN_WARP_ISSUE ? true : lane == 0;
+        if (warp == 8 && issuer_thread)
+            fwd_producer<D, CAUSAL>(p, &tm_q, &tm_k, &tm_v, sQ, sKV, b, lane == 0, abort_flag);
+        else if (warp == 9 && issuer_thread)
+            fwd_mma<D, CAUSAL>(p, tbase, sQ, sKV, b, lane == 0, abort_flag);
     }
 
     tc_fence_before_sync();

@@ -1,7 +1,7 @@
 """Build the sm_100a CUDA library in-tree (``libexact_attn_b200.so`` beside this file).
 
-One translation unit (csrc/attn_api.cu includes every kernel), compiled with
-nvcc for sm_100a only. No GPU is needed to build.
+csrc/attn_api.cu (which includes every kernel) and csrc/attn_noalloc.cu,
+compiled with nvcc for sm_100a only. No GPU is needed to build.
 """
 from __future__ import annotations
 
@@ -41,7 +41,7 @@ def build(force: bool = False, verbose: bool = False) -> str:
     if not force and up_to_date():
         return LIB
     cmd = [NVCC, *FLAGS, "-I", os.path.join(ROOT, "include"), "-I", CSRC,
-           os.path.join(CSRC, "attn_api.cu"), "-o", LIB]
+           os.path.join(CSRC, "attn_api.cu"), os.path.join(CSRC, "attn_noalloc.cu"), "-o", LIB]
     res = subprocess.run(cmd, capture_output=True, text=True)
     if res.returncode != 0:
         sys.stderr.write(res.stdout + res.stderr)

@@ -128,6 +128,8 @@ const char* attn_strerror(attn_status_t s) {
         case ATTN_ERR_ALIGNMENT: return "misaligned pointer (bf16 tensors need 16 bytes, fp32 4)";
         case ATTN_ERR_CUDA: return "CUDA error while launching or running a kernel";
         case ATTN_ERR_TIMEOUT: return "a kernel pipeline wait timed out; outputs are invalid";
+        case ATTN_ERR_SCRATCH_LIMIT:
+            return "partials exceed the library's fixed 32 MiB decode scratch array";
     }
     return "unknown status";
 }

@@ -48,7 +48,8 @@ typedef enum {
     ATTN_ERR_UNSUPPORTED = 2,
     ATTN_ERR_ALIGNMENT = 3,
     ATTN_ERR_CUDA = 4,
-    ATTN_ERR_TIMEOUT = 5
+    ATTN_ERR_TIMEOUT = 5,
+    ATTN_ERR_SCRATCH_LIMIT = 6
 } attn_status_t;
 
 /* Version of this ABI (bumped on any incompatible change). */
@@ -133,6 +134,29 @@ attn_status_t attn_decode_splitkv(const void *q, const void *k, const void *v, v
                                   float *lse, int B, int H, int Nkv, int d, float scale,
                                   int num_splits, void *workspace, size_t workspace_bytes,
                                   void *stream);
+
+/*
+ * Split-KV decode for callers that cannot allocate device memory.
+ *
+ * The pages have no counterpart to this entry point; it exists for library
+ * users. It computes exactly what attn_decode_splitkv computes, with the same
+ * arguments except the workspace: the partials go to a fixed 32 MiB array
+ * owned by this library (one per GPU that loads it, held until the process
+ * exits). It is meant for callers that may not call cudaMalloc or cannot hand
+ * over a device buffer, e.g. code inside an allocator's callbacks or a plugin
+ * whose host framework owns all device memory.
+ *
+ *   Returns ATTN_ERR_SCRATCH_LIMIT, without launching, when the partials
+ *   (attn_decode_workspace_bytes(B, H, d, num_splits) bytes) exceed 32 MiB.
+ *   All calls on a device share the array: calls that overlap on the GPU race
+ *   and must be serialised by the caller. The array keeps the last call's
+ *   contents; none of it needs to start at zero.
+ *   The first call on each device looks up the array's device address
+ *   (cudaGetSymbolAddress); make that first call before any stream capture.
+ */
+attn_status_t attn_decode_splitkv_noalloc(const void *q, const void *k, const void *v, void *o,
+                                          float *lse, int B, int H, int Nkv, int d, float scale,
+                                          int num_splits, void *stream);
 
 /*
  * Synchronises `stream`, then returns and clears the device status word:

@@ -87,10 +87,9 @@ def merge_bytes(w):
 
 # ---------------------------------------------------------------- helpers --
 def dist_env():
-    ws = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
-    return ws, rank, local
+    from exact_io_aware_70_b200.replicas import rank_info
+    r = rank_info()
+    return r.world_size, r.rank, r.local_rank
 
 
 class ClockSampler:
@@ -313,8 +312,9 @@ def run_ours(args):
 
     # ---- inputs resident in HBM (seed offset per rank: each rank its own batch)
     kernels = []
+    from exact_io_aware_70_b200.replicas import max_over_ranks, replica_workload
     if pw:
-        pw_r = dataclasses.replace(pw, seed=pw.seed + 1000 * rank)
+        pw_r = replica_workload(pw, rank)
         q, k, v = make_workload(pw_r, device="cuda")
         o = torch.empty_like(q)
         lse = torch.empty((pw.B, pw.H, pw.Nq), dtype=torch.float32, device=dev)
@@ -325,7 +325,7 @@ def run_ours(args):
                               pw.scale, sp)
         kernels.append(("attn_fwd_sm100", launch_prefill))
     if dw:
-        dw_r = dataclasses.replace(dw, seed=dw.seed + 1000 * rank)
+        dw_r = replica_workload(dw, rank)
         dq, dk, dv = make_workload(dw_r, device="cuda")
         do = torch.empty_like(dq)
         dlse = torch.empty((dw.B, dw.H, 1), dtype=torch.float32, device=dev)
@@ -382,10 +382,7 @@ def run_ours(args):
     total_ms = t_start.elapsed_time(t_end)
     per_kernel_ms = [statistics.mean(ev[s][i].elapsed_time(ev[s][i + 1]) for s in range(K))
                      for i in range(len(kernels))]
-    times = torch.tensor([total_ms] + per_kernel_ms, dtype=torch.float64, device=dev)
-    if ws > 1:
-        dist.all_reduce(times, op=dist.ReduceOp.MAX)
-    total_ms, *per_kernel_ms = times.tolist()
+    total_ms, *per_kernel_ms = max_over_ranks([total_ms] + per_kernel_ms, device=dev)
     kms = dict(zip([n for n, _ in kernels], per_kernel_ms))
 
     # ---- e2e: the same work through the public API from pinned host buffers
@@ -436,10 +433,7 @@ def run_ours(args):
             torch.cuda.synchronize()
             for i in range(len(parts)):
                 acc[i] += ep[i].elapsed_time(ep[i + 1]) / E
-        et = torch.tensor(acc, dtype=torch.float64, device=dev)
-        if ws > 1:
-            dist.all_reduce(et, op=dist.ReduceOp.MAX)
-        acc = et.tolist()
+        acc = max_over_ranks(acc, device=dev)
         if ea.attn_status() != 0:
             raise RuntimeError("device status reported an error in the e2e region")
         e2e = {"h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": sum(acc),

@@ -22,7 +22,9 @@ import ctypes
 import os
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "libexact_attn_b200.so")
+# EXACT_ATTN_LIB may name another build of the same library (e.g. one compiled
+# with different tuning macros); it must exist, there is no fallback either way.
+LIB_PATH = os.environ.get("EXACT_ATTN_LIB") or os.path.join(_HERE, "libexact_attn_b200.so")
 
 if not os.path.exists(LIB_PATH):
     raise ImportError(

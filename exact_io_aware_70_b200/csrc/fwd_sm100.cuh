@@ -77,6 +77,15 @@ struct FwdParams {
 #ifndef EATTN_KV_SLOTS_D128
 #define EATTN_KV_SLOTS_D128 4
 #endif
+// 1: K_j and V_j complete on K_j's full barrier (one wait per K/V pair for
+//    the MMA issuer); 0: each tile has its own full barrier.
+#ifndef EATTN_KV_PAIR_BARRIER
+#define EATTN_KV_PAIR_BARRIER 1
+#endif
+// 1: P is released to the MMA issuer in two halves (p_lo, p_hi); 0: once.
+#ifndef EATTN_SPLIT_P
+#define EATTN_SPLIT_P 1
+#endif
 
 template <int D>
 struct FwdTraits {
@@ -87,6 +96,7 @@ struct FwdTraits {
     static constexpr int kTileBytes = kPanels * kPanelBytes;
     static constexpr int kSlots = (D == 128) ? EATTN_KV_SLOTS_D128 : 8;   // K/V ring depth (tiles)
     static_assert(kSlots >= 2, "the ring holds K_j and V_j at once");
+    static_assert(!EATTN_KV_PAIR_BARRIER || kSlots % 2 == 0, "K/V pairs need an even ring");
     static constexpr int kThreads = 384;                  // 3 warpgroups
     // Registers: the launch gives every thread kLaunchRegs (the build checks
     // ptxas reports exactly that); the softmax warpgroups then grow to
@@ -219,11 +229,17 @@ __device__ void fwd_producer(const FwdParams& p, const CUtensorMap* tq, const CU
                 const uint32_t round = kv_iter / T::kSlots;
                 if (round > 0 && !role_wait(b.kv_empty(slot), (round - 1) & 1, abort_flag))
                     goto fail;
-                mbar_arrive_expect_tx_w(b.kv_full(slot), T::kTileBytes, leader);
+                // with pair barriers, V_j's copy completes on K_j's barrier (slot - 1)
+                const uint32_t fbar =
+                    b.kv_full(EATTN_KV_PAIR_BARRIER && which ? slot - 1 : slot);
+                if (!EATTN_KV_PAIR_BARRIER)
+                    mbar_arrive_expect_tx_w(fbar, T::kTileBytes, leader);
+                else if (which == 0)
+                    mbar_arrive_expect_tx_w(fbar, 2 * T::kTileBytes, leader);
 #pragma unroll
                 for (int pn = 0; pn < T::kPanels; ++pn)
                     tma_load_3d_w(sKV + slot * T::kTileBytes + pn * T::kPanelBytes,
-                                  which ? tv : tk, b.kv_full(slot), pn * 64, j * 128, x.bh, leader);
+                                  which ? tv : tk, fbar, pn * 64, j * 128, x.bh, leader);
                 ++kv_iter;
             }
         }
@@ -235,7 +251,8 @@ fail: {
     volatile int no_abort = 0;
     const uint32_t first = kv_iter > (uint32_t)T::kSlots ? kv_iter - T::kSlots : 0;
     for (uint32_t i = first; i < kv_iter; ++i)
-        mbar_wait(b.kv_full(i % T::kSlots), (i / T::kSlots) & 1, &no_abort, &g_attn_status);
+        if (!EATTN_KV_PAIR_BARRIER || (i % 2) == 0)
+            mbar_wait(b.kv_full(i % T::kSlots), (i / T::kSlots) & 1, &no_abort, &g_attn_status);
     for (int t = 0; t < 2; ++t)
         if (q_issued[t] > 0)
             mbar_wait(b.q_full(t), (q_issued[t] - 1) & 1, &no_abort, &g_attn_status);
@@ -305,24 +322,29 @@ __device__ void fwd_mma(const FwdParams& p, uint32_t tbase, uint32_t sQ, uint32_
             ++kv_iter;
             for (int j = 0; j < x.nmax; ++j) {
                 const uint32_t vslot = kv_iter % T::kSlots;
-                if (!role_wait(b.kv_full(vslot), (kv_iter / T::kSlots) & 1, abort_flag))
-                    goto done;
-                tc_fence_after_sync();
+                if (!EATTN_KV_PAIR_BARRIER) {   // else V_j arrived with K_j
+                    if (!role_wait(b.kv_full(vslot), (kv_iter / T::kSlots) & 1, abort_flag))
+                        goto done;
+                    tc_fence_after_sync();
+                }
                 ++kv_iter;
                 const bool has_next = j + 1 < x.nmax;
                 kslot = kv_iter % T::kSlots;
                 const uint32_t kpar = (kv_iter / T::kSlots) & 1;
                 for (int t = 0; t < 2; ++t) {
                     if (j < x.n[t]) {
-                        if (!role_wait(b.p_lo(t), p_phase[t], abort_flag)) goto done;
+                        if (!role_wait(EATTN_SPLIT_P ? b.p_lo(t) : b.p_hi(t), p_phase[t], abort_flag))
+                            goto done;
                         if (j == 0 && o_use[t] > 0 &&
                             !role_wait(b.o_free(t), (o_use[t] - 1) & 1, abort_flag))
                             goto done;
                         tc_fence_after_sync();
                         fwd_issue_pv<D>(tbase + colO[t], tbase + colS[t], dv0 + vslot * kTileStep,
                                         j > 0, 0, leader);
-                        if (!role_wait(b.p_hi(t), p_phase[t], abort_flag)) goto done;
-                        tc_fence_after_sync();
+                        if (EATTN_SPLIT_P) {
+                            if (!role_wait(b.p_hi(t), p_phase[t], abort_flag)) goto done;
+                            tc_fence_after_sync();
+                        }
                         fwd_issue_pv<D>(tbase + colO[t], tbase + colS[t], dv0 + vslot * kTileStep,
                                         true, 1, leader);
                         p_phase[t] ^= 1;
@@ -430,19 +452,21 @@ __device__ void fwd_softmax(const FwdParams& p, uint32_t tbase, const FwdBars<Fw
                     const f32x2_t xv = f2_fma(
                         f2_pack(__uint_as_float(sr[c]), __uint_as_float(sr[c + 1])), c2x2, nbx2);
                     float e0, e1;
-                    if (kPolyEvery > 0 && (i % (kPolyEvery > 0 ? kPolyEvery : 1)) == kPolyEvery - 1) {
+                    if (kPolyEvery > 0 &&
+                               (i % (kPolyEvery > 0 ? kPolyEvery : 1)) == kPolyEvery - 1) {
                         exp2_poly_pair(xv, e0, e1);
+                        pk[i] = pack_bf16x2(e0, e1);
                     } else {
                         float x0, x1;
                         f2_unpack(xv, x0, x1);
                         e0 = fast_exp2(x0);
                         e1 = fast_exp2(x1);
+                        pk[i] = pack_bf16x2(e0, e1);
                     }
                     if (i & 1)
                         lsum_b = f2_add(lsum_b, f2_pack(e0, e1));
                     else
                         lsum_a = f2_add(lsum_a, f2_pack(e0, e1));
-                    pk[i] = pack_bf16x2(e0, e1);
                 }
                 if (h == 0 && any_need && j > 0) {
                     // Rescale O_t by alpha (1 for rows whose max did not move)
@@ -460,9 +484,11 @@ __device__ void fwd_softmax(const FwdParams& p, uint32_t tbase, const FwdBars<Fw
                     }
                 }
                 tmem_st32(tS + 32 * h, pk);
-                tmem_wait_st();
-                tc_fence_before_sync();
-                mbar_arrive(h == 0 ? bar_plo : bar_phi);
+                if (EATTN_SPLIT_P || h == 1) {
+                    tmem_wait_st();
+                    tc_fence_before_sync();
+                    mbar_arrive(h == 0 ? bar_plo : bar_phi);
+                }
             }
             float la0, la1, lb0, lb1;
             f2_unpack(lsum_a, la0, la1);

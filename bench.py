@@ -160,15 +160,20 @@ def kernel_source_hash():
 
 def recorded_traffic():
     """Per-launch DRAM traffic from the committed ncu summary, if taken on this source."""
-    path = os.path.join(ROOT, "profiles", "dram_traffic.json")
+    path = os.path.join(ROOT, "profiles", "dram_traffic.md")
     try:
         with open(path) as fh:
-            rec = json.load(fh)
-    except (OSError, ValueError):
+            text = fh.read()
+    except OSError:
         return {}
-    if rec.get("source_hash") != kernel_source_hash():
+    import re
+    m = re.search(r"source_hash:\s*([0-9a-f]+)", text)
+    if not m or m.group(1) != kernel_source_hash():
         return {}
-    return rec.get("per_launch_bytes", {})
+    out = {}
+    for row in re.findall(r"^\|\s*(attn_\w+)\s*\|\s*\w+\s*\|\s*(\d+)\s*\|", text, re.M):
+        out[row[0]] = int(row[1])
+    return out
 
 
 # ------------------------------------------------------------ CPU oracle --

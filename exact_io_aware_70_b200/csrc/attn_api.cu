@@ -23,6 +23,23 @@ __device__ unsigned g_attn_status = 0;
 
 using namespace eattn;
 
+namespace eattn {
+// Waits on an mbarrier that nothing ever arrives on, through the same bounded
+// wait every pipeline kernel uses, so the give-up path can be exercised
+// without faulting or hanging the GPU.
+__global__ void attn_wait_selftest_kernel(unsigned long long limit_ns) {
+    __shared__ __align__(8) uint64_t bar;
+    __shared__ int abort_flag;
+    if (threadIdx.x == 0) {
+        mbar_init(smem_addr(&bar), 1);
+        abort_flag = 0;
+        fence_mbar_init();
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) mbar_wait_limit(smem_addr(&bar), 0, &abort_flag, &g_attn_status, limit_ns);
+}
+}  // namespace eattn
+
 namespace {
 
 constexpr int kAbiVersion = 1;
@@ -252,6 +269,13 @@ attn_status_t attn_decode_splitkv(const void* q, const void* k, const void* v, v
                                            num_splits, stream);
     if (s != ATTN_OK) return s;
     return attn_lse_merge(o_part, lse_part, o, lse, B, H, num_splits, d, stream);
+}
+
+attn_status_t attn_selftest_wait_timeout(unsigned limit_us, void* stream) {
+    if (limit_us < 1 || limit_us > 1000000) return ATTN_ERR_INVALID_ARG;
+    attn_wait_selftest_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(
+        (unsigned long long)limit_us * 1000ull);
+    return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
 
 attn_status_t attn_status(void* stream) {

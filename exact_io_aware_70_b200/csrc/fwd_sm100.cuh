@@ -48,9 +48,11 @@
 //     out of the polynomial as about 2^-125 rather than 0: negligible next to
 //     the row sum (at least 1 once a row has seen a visible key), and rows with
 //     no visible key at all are set to O = 0, LSE = -inf in the epilogue.
-//   * P_t is handed to the MMA warp in two halves (keys 0-63, then 64-127),
-//     so the first half of O_t += P_t V_j runs while the second half of the
-//     exponentials is still being computed.
+//   * P_t is handed to the MMA warp once per step (EATTN_SPLIT_P=1 hands it
+//     over in two halves so the first half of O_t += P_t V_j can start early;
+//     that costs the MMA issuer one more barrier check per tile and step and
+//     measured slower). K_j and V_j complete on one barrier, and each Q tile is
+//     released to the producer right after its last S product of the unit.
 //   * Tensor memory columns: S0 [0,128), S1 [128,256), O0 [256,256+d),
 //     O1 [256+d, 256+2d).
 #pragma once
@@ -84,7 +86,7 @@ struct FwdParams {
 #endif
 // 1: P is released to the MMA issuer in two halves (p_lo, p_hi); 0: once.
 #ifndef EATTN_SPLIT_P
-#define EATTN_SPLIT_P 1
+#define EATTN_SPLIT_P 0
 #endif
 
 template <int D>
@@ -317,6 +319,8 @@ __device__ void fwd_mma(const FwdParams& p, uint32_t tbase, uint32_t sQ, uint32_
                     fwd_issue_s<D>(tbase + colS[t], dq0 + t * kTileStep, dk0 + kslot * kTileStep,
                                    leader);
                     mma_commit_w(b.s_full(t), leader);
+                    // Q_t's last use in this unit: let the producer refill it now
+                    if (x.n[t] == 1) mma_commit_w(b.q_empty(t), leader);
                 }
             mma_commit_w(b.kv_empty(kslot), leader);
             ++kv_iter;
@@ -359,6 +363,7 @@ __device__ void fwd_mma(const FwdParams& p, uint32_t tbase, uint32_t sQ, uint32_
                         fwd_issue_s<D>(tbase + colS[t], dq0 + t * kTileStep,
                                        dk0 + kslot * kTileStep, leader);
                         mma_commit_w(b.s_full(t), leader);
+                        if (j + 2 == x.n[t]) mma_commit_w(b.q_empty(t), leader);
                     }
                 }
                 if (has_next) {
@@ -367,8 +372,9 @@ __device__ void fwd_mma(const FwdParams& p, uint32_t tbase, uint32_t sQ, uint32_
                 }
             }
         }
-        mma_commit_w(b.q_empty(0), leader);
-        mma_commit_w(b.q_empty(1), leader);
+        // Q tiles without any S product in this unit are released here
+        for (int t = 0; t < 2; ++t)
+            if (x.n[t] == 0) mma_commit_w(b.q_empty(t), leader);
         ++q_use;
         for (int t = 0; t < 2; ++t)
             if (x.n[t] > 0) ++o_use[t];

@@ -65,19 +65,25 @@ __device__ __forceinline__ bool mbar_test(uint32_t bar, uint32_t parity) {
 
 // Bounded wait for the phase of `bar` with the given parity to complete.
 // `abort_flag` is the CTA's shared abort word. Returns false on give-up.
-__device__ __forceinline__ bool mbar_wait_slow(uint32_t bar, uint32_t parity,
-                                            volatile int* abort_flag, unsigned* status) {
+__device__ __forceinline__ bool mbar_wait_limit(uint32_t bar, uint32_t parity,
+                                                volatile int* abort_flag, unsigned* status,
+                                                unsigned long long limit_ns) {
     const unsigned long long t0 = global_timer_ns();
     for (unsigned polls = 0; polls < kWaitMaxPolls; ++polls) {
         if (mbar_test(bar, parity)) return true;
         if ((polls & 31u) == 31u) {
             if (*abort_flag) return false;
-            if (global_timer_ns() - t0 > kWaitLimitNs) break;
+            if (global_timer_ns() - t0 > limit_ns) break;
         }
     }
     *abort_flag = 1;
     atomicOr(status, kDevErrTimeout);
     return false;
+}
+
+__device__ __forceinline__ bool mbar_wait_slow(uint32_t bar, uint32_t parity,
+                                               volatile int* abort_flag, unsigned* status) {
+    return mbar_wait_limit(bar, parity, abort_flag, status, kWaitLimitNs);
 }
 
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag,

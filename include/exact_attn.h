@@ -166,6 +166,16 @@ attn_status_t attn_decode_splitkv_noalloc(const void *q, const void *k, const vo
  */
 attn_status_t attn_status(void *stream);
 
+/*
+ * Diagnostic for the failure-detection path: enqueues a one-block kernel that
+ * waits on a barrier nothing ever completes, through the same bounded wait the
+ * pipeline kernels use, with a limit of `limit_us` microseconds
+ * (1 <= limit_us <= 1000000). The kernel gives up, records a timeout and
+ * exits; the next attn_status() on the stream returns ATTN_ERR_TIMEOUT, and the
+ * CUDA context stays usable. No counterpart on the pages (library testing aid).
+ */
+attn_status_t attn_selftest_wait_timeout(unsigned limit_us, void *stream);
+
 /* A static, human-readable description of a status code. */
 const char *attn_strerror(attn_status_t status);
 

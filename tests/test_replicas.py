@@ -39,7 +39,7 @@ def _worker(rank, world, port, out):
 
 def test_two_gloo_ranks():
     port = 29500 + os.getpid() % 1000
-    with mp.Manager() as m:
+    with mp.get_context("spawn").Manager() as m:
         out = m.dict()
         mp.start_processes(_worker, args=(2, port, out), nprocs=2, start_method="spawn")
         r0, r1 = out[0], out[1]

@@ -40,13 +40,14 @@
 //     LSE = ln 2 * (m + log2 l)).
 //   * Exponentials are base 2 with log2(e) folded into the scale, computed
 //     with MUFU ex2 on pairs prepared by sm_100's packed f32x2 FMA; the row
-//     max uses the three-input max. Optionally (EATTN_POLY_EVERY = k > 0) one
-//     pair in every k is exponentiated on the FMA pipe (exp2_poly_pair)
-//     instead; measured on B200 this is slower at every k tried (2, 3, 4, 8)
-//     because the softmax is issue-bound rather than MUFU-bound once the
-//     pairs are packed, so it is off by default. A masked (-inf) score comes
-//     out of the polynomial as about 2^-125 rather than 0: negligible next to
-//     the row sum (at least 1 once a row has seen a visible key), and rows with
+//     max uses the three-input max. A fraction of the pairs can instead be
+//     exponentiated on the FMA pipe (exp2_poly_pair, kPolyEvery<D>); measured
+//     on B200 it is slower at every fraction tried, at d=128 (MUFU and tensor
+//     core need the same cycles per step) and at d=64 (short sequences are
+//     latency-bound), so it is off by default. A masked
+//     (-inf) score comes out of the polynomial as about 2^-125 rather than 0:
+//     negligible next to the row sum (at least 1 once a row has seen a
+//     visible key), and rows with
 //     no visible key at all are set to O = 0, LSE = -inf in the epilogue.
 //   * P_t is handed to the MMA warp once per step (EATTN_SPLIT_P=1 hands it
 //     over in two halves so the first half of O_t += P_t V_j can start early;
@@ -81,6 +82,11 @@ struct FwdParams {
 #endif
 // 1: K_j and V_j complete on K_j's full barrier (one wait per K/V pair for
 //    the MMA issuer); 0: each tile has its own full barrier.
+// 1: TMA loads carry L2 policies: K/V tiles (re-read by every query block of
+//    their head) evict-last, Q tiles (read by one CTA) evict-first.
+#ifndef EATTN_FWD_L2_HINTS
+#define EATTN_FWD_L2_HINTS 1
+#endif
 #ifndef EATTN_KV_PAIR_BARRIER
 #define EATTN_KV_PAIR_BARRIER 1
 #endif
@@ -117,11 +123,16 @@ struct FwdTraits {
     static constexpr uint32_t kColO0 = 256, kColO1 = 256 + D;
 };
 
-#ifndef EATTN_POLY_EVERY
-#define EATTN_POLY_EVERY 0
+// One exponent pair in every kPolyEvery<D> goes to the FMA-pipe polynomial
+// (0: none, the measured-best setting for both head dims).
+#ifndef EATTN_POLY_EVERY_D128
+#define EATTN_POLY_EVERY_D128 0
 #endif
-// One exponent pair in every kPolyEvery goes to the FMA-pipe polynomial (0: none).
-constexpr int kPolyEvery = EATTN_POLY_EVERY;
+#ifndef EATTN_POLY_EVERY_D64
+#define EATTN_POLY_EVERY_D64 0
+#endif
+template <int D>
+constexpr int kPolyEvery = (D == 128) ? EATTN_POLY_EVERY_D128 : EATTN_POLY_EVERY_D64;
 
 // Unit handled by this CTA in round r (snake order), or -1 past the end.
 __device__ __forceinline__ int fwd_unit_of_round(int r, int num_units) {
@@ -210,6 +221,8 @@ __device__ void fwd_producer(const FwdParams& p, const CUtensorMap* tq, const CU
                              const FwdBars<FwdTraits<D>::kSlots>& b, uint32_t leader,
                              volatile int* abort_flag) {
     using T = FwdTraits<D>;
+    const uint64_t pol_q = l2_policy_evict_first();
+    const uint64_t pol_kv = l2_policy_evict_last();
     uint32_t kv_iter = 0;
     uint32_t q_issued[2] = {0, 0};
     FWD_FOR_EACH_UNIT(u, p) {
@@ -220,8 +233,13 @@ __device__ void fwd_producer(const FwdParams& p, const CUtensorMap* tq, const CU
             mbar_arrive_expect_tx_w(b.q_full(t), T::kTileBytes, leader);
 #pragma unroll
             for (int pn = 0; pn < T::kPanels; ++pn)
-                tma_load_3d_w(sQ + t * T::kTileBytes + pn * T::kPanelBytes, tq, b.q_full(t),
-                              pn * 64, x.qb * 256 + t * 128, x.bh, leader);
+                if (EATTN_FWD_L2_HINTS)
+                    tma_load_3d_hint_w(sQ + t * T::kTileBytes + pn * T::kPanelBytes, tq,
+                                       b.q_full(t), pn * 64, x.qb * 256 + t * 128, x.bh, pol_q,
+                                       leader);
+                else
+                    tma_load_3d_w(sQ + t * T::kTileBytes + pn * T::kPanelBytes, tq, b.q_full(t),
+                                  pn * 64, x.qb * 256 + t * 128, x.bh, leader);
             ++q_issued[t];
         }
         for (int j = 0; j < x.nmax; ++j) {
@@ -240,8 +258,13 @@ __device__ void fwd_producer(const FwdParams& p, const CUtensorMap* tq, const CU
                     mbar_arrive_expect_tx_w(fbar, 2 * T::kTileBytes, leader);
 #pragma unroll
                 for (int pn = 0; pn < T::kPanels; ++pn)
-                    tma_load_3d_w(sKV + slot * T::kTileBytes + pn * T::kPanelBytes,
-                                  which ? tv : tk, fbar, pn * 64, j * 128, x.bh, leader);
+                    if (EATTN_FWD_L2_HINTS)
+                        tma_load_3d_hint_w(sKV + slot * T::kTileBytes + pn * T::kPanelBytes,
+                                           which ? tv : tk, fbar, pn * 64, j * 128, x.bh, pol_kv,
+                                           leader);
+                    else
+                        tma_load_3d_w(sKV + slot * T::kTileBytes + pn * T::kPanelBytes,
+                                      which ? tv : tk, fbar, pn * 64, j * 128, x.bh, leader);
                 ++kv_iter;
             }
         }
@@ -458,8 +481,8 @@ __device__ void fwd_softmax(const FwdParams& p, uint32_t tbase, const FwdBars<Fw
                     const f32x2_t xv = f2_fma(
                         f2_pack(__uint_as_float(sr[c]), __uint_as_float(sr[c + 1])), c2x2, nbx2);
                     float e0, e1;
-                    if (kPolyEvery > 0 &&
-                               (i % (kPolyEvery > 0 ? kPolyEvery : 1)) == kPolyEvery - 1) {
+                    if (kPolyEvery<D> > 0 &&
+                               (i % (kPolyEvery<D> > 0 ? kPolyEvery<D> : 1)) == kPolyEvery<D> - 1) {
                         exp2_poly_pair(xv, e0, e1);
                         pk[i] = pack_bf16x2(e0, e1);
                     } else {

@@ -126,6 +126,33 @@ __device__ __forceinline__ void mbar_arrive_expect_tx_w(uint32_t bar, uint32_t b
         : "memory");
 }
 
+// L2 eviction policies (createpolicy): data read once is marked evict-first,
+// data re-read by other CTAs evict-last.
+__device__ __forceinline__ uint64_t l2_policy_evict_first() {
+    uint64_t pol;
+    asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
+    return pol;
+}
+__device__ __forceinline__ uint64_t l2_policy_evict_last() {
+    uint64_t pol;
+    asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(pol));
+    return pol;
+}
+
+// tma_load_3d_w with an L2 cache policy.
+__device__ __forceinline__ void tma_load_3d_hint_w(uint32_t dst, const CUtensorMap* map,
+                                                   uint32_t bar, int x, int y, int z,
+                                                   uint64_t policy, uint32_t leader) {
+    asm volatile(
+        "{\n\t.reg .pred e;\n\t"
+        "setp.ne.b32 e, %6, 0;\n\t"
+        "@e cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+        ".L2::cache_hint [%0], [%1, {%2, %3, %4}], [%5], %7;\n\t}" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(bar), "r"(leader),
+        "l"(policy)
+        : "memory");
+}
+
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* map) {
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }

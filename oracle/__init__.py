@@ -46,6 +46,10 @@ class Oracle:
                                                     ctypes.c_double, _c_long, _dp, _dp]
         lib.oracle_lse_merge_f64.argtypes = [_dp, _dp, _c_long, _c_long, _dp, _dp]
         lib.oracle_lse_merge_f32in.argtypes = [_fp, _fp, _c_long, _c_long, _c_long, _dp, _dp]
+        _i32p = ctypes.POINTER(ctypes.c_int32)
+        lib.oracle_decode_paged_bf16.argtypes = [_u16p, _u16p, _u16p, _i32p, _i32p, _c_long,
+                                                 _c_long, _c_long, _c_long, _c_long, _c_long,
+                                                 ctypes.c_double, _dp, _dp]
         lib.oracle_num_threads.restype = ctypes.c_int
         lib.oracle_set_num_threads.argtypes = [ctypes.c_int]
         self.lib = lib
@@ -111,6 +115,29 @@ class Oracle:
             raise RuntimeError("oracle_decode_partials_bf16 failed")
         return o, lse
 
+    def decode_paged_bf16(self, q_bits, k_cache_bits, v_cache_bits, block_table, seq_lens,
+                          scale: float):
+        """q [B,H,d]; caches [num_pages,H,page_size,d] uint16; block_table [B,max_pages] int32;
+        seq_lens [B] int32 -> (O [B,H,d] f64, LSE [B,H] f64)."""
+        q = np.ascontiguousarray(q_bits, dtype=np.uint16)
+        kc = np.ascontiguousarray(k_cache_bits, dtype=np.uint16)
+        vc = np.ascontiguousarray(v_cache_bits, dtype=np.uint16)
+        bt = np.ascontiguousarray(block_table, dtype=np.int32)
+        sl = np.ascontiguousarray(seq_lens, dtype=np.int32)
+        B, H, d = q.shape
+        num_pages, H2, page_size, d2 = kc.shape
+        assert H2 == H and d2 == d and vc.shape == kc.shape and bt.shape[0] == B
+        o = np.zeros((B, H, d))
+        lse = np.zeros((B, H))
+        i32 = ctypes.POINTER(ctypes.c_int32)
+        rc = self.lib.oracle_decode_paged_bf16(_ptr(q, _u16p), _ptr(kc, _u16p), _ptr(vc, _u16p),
+                                               _ptr(bt, i32), _ptr(sl, i32), B, H, d, page_size,
+                                               bt.shape[1], num_pages, float(scale),
+                                               _ptr(o, _dp), _ptr(lse, _dp))
+        if rc:
+            raise RuntimeError("oracle_decode_paged_bf16 failed")
+        return o, lse
+
     def lse_merge_f64(self, o_part, lse_part):
         o_part = np.ascontiguousarray(o_part, dtype=np.float64)
         lse_part = np.ascontiguousarray(lse_part, dtype=np.float64)
@@ -155,7 +182,7 @@ def get() -> Oracle:
 
 
 def build_mutant(n: int, out_dir: str) -> Oracle:
-    """A copy of the oracle with planted mistake ``n`` (1..9), for the pin tests."""
+    """A copy of the oracle with planted mistake ``n`` (1..11), for the pin tests."""
     out = os.path.join(out_dir, f"liboracle_mutant{n}.so")
     _build.build(out=out, mutant=n, force=True)
     return Oracle(out)

@@ -338,6 +338,65 @@ int oracle_lse_merge_f32in(const float *o_part, const float *lse_part, long BH,
     return rc;
 }
 
+/*
+ * Paged-KV decode: one query row per (b, h) attends to the seq_lens[b] cached
+ * tokens of sequence b, stored in fixed-size pages. Token j of sequence b lives
+ * in physical page block_table[b][j / page_size], slot j % page_size; a page
+ * holds page_size tokens of every head, laid out [num_pages][H][page_size][d].
+ * (The serving variant of split-KV decode, "paged variants for decode",
+ * mantramindai "Versions"; the layout is this library's reading: the pages give
+ * none.) The result is the plain definition over the gathered keys; a
+ * sequence with no token gives O = 0, LSE = -inf.
+ *   q [B, H, d]; k_cache, v_cache [num_pages, H, page_size, d] (bf16 bits);
+ *   block_table [B, max_pages]; seq_lens [B]; o [B, H, d]; lse [B, H].
+ * Returns -1 on an invalid size or a table entry outside [0, num_pages).
+ */
+int oracle_decode_paged_bf16(const uint16_t *q, const uint16_t *k_cache, const uint16_t *v_cache,
+                             const int32_t *block_table, const int32_t *seq_lens, long B, long H,
+                             long d, long page_size, long max_pages, long num_pages,
+                             double scale, double *o, double *lse) {
+    if (B < 0 || H < 0 || d <= 0 || page_size <= 0 || max_pages <= 0 || num_pages <= 0) return -1;
+    for (long b = 0; b < B; ++b) {
+        long n = seq_lens[b];
+        if (n < 0 || n > max_pages * page_size) return -1;
+#if ORACLE_MUTANT == 11 /* reads one token past the sequence */
+        if (n < max_pages * page_size) n += 1;
+#endif
+        double *kh = (double *)malloc((size_t)((n > 0 ? n : 1) * d) * sizeof(double));
+        double *vh = (double *)malloc((size_t)((n > 0 ? n : 1) * d) * sizeof(double));
+        double *qh = (double *)malloc((size_t)d * sizeof(double));
+        int rc = (kh && vh && qh) ? 0 : -1;
+        for (long h = 0; rc == 0 && h < H; ++h) {
+            for (long j = 0; j < n; ++j) {
+#if ORACLE_MUTANT == 10 /* ignores the block table (logical page = physical page) */
+                long page = j / page_size;
+#else
+                long page = block_table[b * max_pages + j / page_size];
+#endif
+                if (page < 0 || page >= num_pages) { rc = -1; break; }
+                const uint16_t *kr = k_cache + ((page * H + h) * page_size + j % page_size) * d;
+                const uint16_t *vr = v_cache + ((page * H + h) * page_size + j % page_size) * d;
+                for (long c = 0; c < d; ++c) {
+                    kh[j * d + c] = bf16_to_double(kr[c]);
+                    vh[j * d + c] = bf16_to_double(vr[c]);
+                }
+            }
+            if (rc) break;
+            for (long c = 0; c < d; ++c) qh[c] = bf16_to_double(q[(b * H + h) * d + c]);
+            if (n == 0) {
+                for (long c = 0; c < d; ++c) o[(b * H + h) * d + c] = 0.0;
+                lse[b * H + h] = -INFINITY;
+                continue;
+            }
+            rc = oracle_attn_head_f64(qh, kh, vh, 1, n, d, 0, scale, o + (b * H + h) * d,
+                                      lse + b * H + h, NULL);
+        }
+        free(kh); free(vh); free(qh);
+        if (rc) return rc;
+    }
+    return 0;
+}
+
 /* number of OpenMP threads the oracle will use (1 without OpenMP) */
 int oracle_num_threads(void) {
 #ifdef _OPENMP

@@ -302,9 +302,70 @@ def pin_bf16_entry(orc):
     _close(o_w[0], [1.0, -2.0, 0.15625], 0.0, "bf16 widening")
 
 
+# ---------------------------------------------------------------------------
+# 7. Paged-KV decode (the serving variant of split-KV decode)
+# ---------------------------------------------------------------------------
+def _paged_layout(k, v, lens, page_size, perm_seed=None):
+    """Scatter contiguous K, V [B,H,L,d] (bf16 bits) into pages [P,H,page_size,d]
+    with a block table; physical page order optionally shuffled."""
+    B, H, L, d = k.shape
+    max_pages = L // page_size
+    num_pages = B * max_pages
+    order = np.arange(num_pages)
+    if perm_seed is not None:
+        order = np.random.default_rng(perm_seed).permutation(num_pages)
+    table = order.reshape(B, max_pages).astype(np.int32)
+    kc = np.zeros((num_pages, H, page_size, d), dtype=np.uint16)
+    vc = np.zeros_like(kc)
+    for b in range(B):
+        for i in range(max_pages):
+            kc[table[b, i]] = k[b, :, i * page_size:(i + 1) * page_size]
+            vc[table[b, i]] = v[b, :, i * page_size:(i + 1) * page_size]
+    return kc, vc, table, np.asarray(lens, dtype=np.int32)
+
+
+def pin_paged_matches_contiguous(orc):
+    """Any page placement gives the attention of the row over its first seq_len keys."""
+    from seeded_inputs import bf16_bits, make_qkv
+    B, H, L, d, ps = 3, 2, 64, 8, 16
+    q, k, v = make_qkv(B, H, 1, L, d, seed=34)
+    qb, kb, vb = bf16_bits(q), bf16_bits(k), bf16_bits(v)
+    lens = [37, 64, 1]
+    for perm in (None, 35):
+        kc, vc, table, sl = _paged_layout(kb, vb, lens, ps, perm)
+        o, lse = orc.decode_paged_bf16(qb[:, :, 0], kc, vc, table, sl, 0.3)
+        for b in range(B):
+            for h in range(H):
+                n = lens[b]
+                ro, rl = orc.attn_rows_bf16(qb[b, h], kb[b, h, :n], vb[b, h, :n], [0], False, 0.3)
+                _close(o[b, h], ro[0], 1e-12, f"paged O b{b} h{h} perm{perm}")
+                _close(lse[b, h], rl[0], 1e-12, f"paged LSE b{b} h{h} perm{perm}")
+
+
+def pin_paged_golden(orc):
+    """Hand-derived: 3 tokens in pages stored in swapped physical order, q = 0, so
+    O is the mean of the 3 visible values and LSE = ln 3; the fourth slot holds a
+    value that must never be read. A second sequence of length 0 gives 0, -inf."""
+    one = np.float32(1.0)
+    def bits(x):
+        return np.array(x, dtype=np.float32).view(np.uint32).astype(np.uint64).__rshift__(16).astype(np.uint16)
+    q = bits(np.zeros((2, 1, 2)))
+    kc = bits(np.zeros((2, 1, 2, 2)))
+    # physical page 1 = logical page 0 (tokens 0, 1); physical page 0 = logical page 1 (token 2, unused slot)
+    vc = bits(np.array([[[[6.0, 3.0], [1000.0, 1000.0]]], [[[0.0, 3.0], [3.0, 0.0]]]], dtype=np.float32))
+    table = np.array([[1, 0], [0, 1]], dtype=np.int32)
+    lens = np.array([3, 0], dtype=np.int32)
+    o, lse = orc.decode_paged_bf16(q, kc, vc, table, lens, float(one))
+    _close(o[0, 0], [3.0, 2.0], 1e-12, "paged golden O")      # mean of (0,3), (3,0), (6,3)
+    _close(lse[0, 0], math.log(3.0), 1e-12, "paged golden LSE")
+    _close(o[1, 0], [0.0, 0.0], 0.0, "empty sequence O")
+    assert lse[1, 0] == -math.inf
+
+
 ALL_PINS = [
     pin_worked_example, pin_golden_cases, pin_probabilities, pin_constant_values,
     pin_identical_keys, pin_zero_query, pin_causal_first_row, pin_key_permutation,
     pin_value_linearity, pin_causal_is_truncation, pin_torch_sdpa, pin_merge_any_chunking,
     pin_partials_are_chunk_attention, pin_merge_batched_matches_single, pin_bf16_entry,
+    pin_paged_matches_contiguous, pin_paged_golden,
 ]

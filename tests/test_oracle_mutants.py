@@ -3,7 +3,8 @@
 The oracle source has ORACLE_MUTANT switches, each planting one plausible bug
 (dropped scale, wrong key index, off-by-one or mis-aligned causal mask, sign
 error in the exponent, dropped normalisation, LSE without the max term,
-transposed V, unnormalised merge weights). Building each variant and running
+transposed V, unnormalised merge weights, a paged decode that ignores its block
+table or reads past the sequence). Building each variant and running
 the pins shows the pins would notice that mistake in the real oracle.
 """
 import pytest
@@ -21,6 +22,8 @@ MUTANTS = {
     7: "LSE without the max term",
     8: "transposed V operand",
     9: "merge weights not normalised",
+    10: "paged decode ignores the block table",
+    11: "paged decode reads one token past the sequence",
 }
 
 
@@ -31,6 +34,6 @@ def test_mutant_is_caught(tmp_path, n):
     for pin in oracle_pins.ALL_PINS:
         try:
             pin(bad)
-        except AssertionError:
+        except (AssertionError, RuntimeError):   # a wrong answer or a refused input
             failed.append(pin.__name__)
     assert failed, f"mutant {n} ({MUTANTS[n]}) passed every pin"

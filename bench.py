@@ -306,10 +306,16 @@ def run_ours(args):
     sp = stream.cuda_stream
     L = ea.lib
 
+    paged = args.workload == "decode_32k_paged"
     if args.workload == "step":
         pw, dw = PREFILL, DECODE
     elif args.workload in ("prefill_8k", "prefill_16k", "gpt2_1k", "tiny"):
         pw, dw = WORKLOADS[args.workload], None
+    elif paged:
+        from seeded_inputs import PAGED_DECODE as PD
+        pw = None
+        dw = dataclasses.replace(DECODE, name=PD["name"], B=PD["B"], H=PD["H"], Nkv=PD["seq_len"],
+                                 d=PD["d"], num_splits=PD["num_splits"], seed=PD["seed"])
     else:
         pw, dw = None, WORKLOADS[args.workload]
     pw = _maybe_batch(pw, args.batch) if pw else None
@@ -329,7 +335,32 @@ def run_ours(args):
                               lse.data_ptr(), pw.B, pw.H, pw.Nq, pw.Nkv, pw.d, int(pw.causal),
                               pw.scale, sp)
         kernels.append(("attn_fwd_sm100", launch_prefill))
-    if dw:
+    if dw and paged:
+        from seeded_inputs import PAGED_DECODE as PD, make_paged_cache
+        dw_r = replica_workload(dw, rank)
+        dq, dk, dv, dtable, dlens = make_paged_cache(dw.B, dw.H, [dw.Nkv] * dw.B, dw.d,
+                                                     PD["page_size"], dw_r.seed, device="cuda")
+        do = torch.empty_like(dq)
+        dlse = torch.empty((dw.B, dw.H, 1), dtype=torch.float32, device=dev)
+        S = dw.num_splits
+        work = torch.empty(ea.attn_decode_workspace_bytes(dw.B, dw.H, dw.d, S), dtype=torch.uint8,
+                           device=dev)
+        o_bytes = ((dw.B * dw.H * S * dw.d * 4 + 255) // 256) * 256
+        o_part = work.data_ptr()
+        lse_part = work.data_ptr() + o_bytes
+        npages, ps = dk.shape[0], PD["page_size"]
+
+        def launch_partials():
+            return L.attn_decode_paged_partials(dq.data_ptr(), dk.data_ptr(), dv.data_ptr(),
+                                                dtable.data_ptr(), dlens.data_ptr(), o_part,
+                                                lse_part, dw.B, dw.H, dw.d, ps, dtable.shape[1],
+                                                npages, dw.scale, S, sp)
+
+        def launch_merge():
+            return L.attn_lse_merge(o_part, lse_part, do.data_ptr(), dlse.data_ptr(), dw.B, dw.H,
+                                    S, dw.d, sp)
+        kernels += [("attn_decode_partials", launch_partials), ("attn_lse_merge", launch_merge)]
+    elif dw:
         dw_r = replica_workload(dw, rank)
         dq, dk, dv = make_workload(dw_r, device="cuda")
         do = torch.empty_like(dq)
@@ -419,7 +450,10 @@ def run_ours(args):
             dq.copy_(hdq, non_blocking=True)
             dk.copy_(hdk, non_blocking=True)
             dv.copy_(hdv, non_blocking=True)
-            ea.attn_decode_splitkv(dq, dk, dv, do, dlse, dw.scale, S, work)
+            if paged:
+                ea.attn_decode_paged(dq, dk, dv, dtable, dlens, do, dlse, dw.scale, S, work)
+            else:
+                ea.attn_decode_splitkv(dq, dk, dv, do, dlse, dw.scale, S, work)
             hdo.copy_(do, non_blocking=True)
             hdl.copy_(dlse, non_blocking=True)
 
@@ -525,7 +559,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="step",
-                    choices=["step", "prefill_8k", "prefill_16k", "gpt2_1k", "tiny", "decode_32k"],
+                    choices=["step", "prefill_8k", "prefill_16k", "gpt2_1k", "tiny", "decode_32k",
+                             "decode_32k_paged"],
                     help="step = prefill_8k + decode_32k (the default bench line)")
     ap.add_argument("--batch", type=int, default=0,
                     help="override the batch size (small profiling captures only)")

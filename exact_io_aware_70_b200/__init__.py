@@ -53,6 +53,10 @@ lib.attn_decode_workspace_bytes.argtypes = [_i, _i, _i, _i]
 lib.attn_decode_splitkv.restype = _i
 lib.attn_decode_splitkv.argtypes = [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _f, _i, _vp, _sz,
                                     _vp]
+lib.attn_decode_paged_partials.restype = _i
+lib.attn_decode_paged_partials.argtypes = [_vp] * 7 + [_i] * 6 + [_f, _i, _vp]
+lib.attn_decode_paged.restype = _i
+lib.attn_decode_paged.argtypes = [_vp] * 7 + [_i] * 6 + [_f, _i, _vp, _sz, _vp]
 lib.attn_status.restype = _i
 lib.attn_status.argtypes = [_vp]
 
@@ -62,6 +66,8 @@ ATTN_ERR_UNSUPPORTED = 2
 ATTN_ERR_ALIGNMENT = 3
 ATTN_ERR_CUDA = 4
 ATTN_ERR_TIMEOUT = 5
+ATTN_ERR_SCRATCH_LIMIT = 6
+ATTN_ERR_BAD_INDEX = 7
 
 
 class AttnError(RuntimeError):
@@ -157,6 +163,29 @@ def attn_decode_splitkv(q, k, v, o, lse, scale: float, num_splits: int, workspac
                                    _tensor(lse, torch.float32, "lse"), B, H, Nkv, d, float(scale),
                                    int(num_splits), _tensor(workspace, torch.uint8, "workspace"),
                                    workspace.numel(), _stream(stream)), "attn_decode_splitkv")
+
+
+def attn_decode_paged(q, k_cache, v_cache, block_table, seq_lens, o, lse, scale: float,
+                      num_splits: int, workspace, num_pages: int | None = None,
+                      stream=None) -> None:
+    """Paged-KV split-KV decode. q [B,H,1,d]; caches [num_pages,H,page_size,d] bf16;
+    block_table [B,max_pages] int32; seq_lens [B] int32; o [B,H,1,d]; lse [B,H,1]."""
+    import torch
+    B, H, one, d = q.shape
+    P, H2, page_size, d2 = k_cache.shape
+    if one != 1 or H2 != H or d2 != d or tuple(v_cache.shape) != tuple(k_cache.shape) \
+            or block_table.shape[0] != B or tuple(seq_lens.shape) != (B,):
+        raise ValueError("attn_decode_paged: inconsistent shapes")
+    _check(lib.attn_decode_paged(_tensor(q, torch.bfloat16, "q"),
+                                 _tensor(k_cache, torch.bfloat16, "k_cache"),
+                                 _tensor(v_cache, torch.bfloat16, "v_cache"),
+                                 _tensor(block_table, torch.int32, "block_table"),
+                                 _tensor(seq_lens, torch.int32, "seq_lens"),
+                                 _tensor(o, torch.bfloat16, "o"), _tensor(lse, torch.float32, "lse"),
+                                 B, H, d, page_size, block_table.shape[1],
+                                 P if num_pages is None else int(num_pages), float(scale),
+                                 int(num_splits), _tensor(workspace, torch.uint8, "workspace"),
+                                 workspace.numel(), _stream(stream)), "attn_decode_paged")
 
 
 def attn_status(stream=None) -> int:

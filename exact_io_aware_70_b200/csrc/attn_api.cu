@@ -147,6 +147,8 @@ const char* attn_strerror(attn_status_t s) {
         case ATTN_ERR_TIMEOUT: return "a kernel pipeline wait timed out; outputs are invalid";
         case ATTN_ERR_SCRATCH_LIMIT:
             return "partials exceed the library's fixed 32 MiB decode scratch array";
+        case ATTN_ERR_BAD_INDEX:
+            return "a block-table entry or sequence length was out of range; those keys were skipped";
     }
     return "unknown status";
 }
@@ -212,11 +214,87 @@ attn_status_t attn_decode_partials(const void* q, const void* k, const void* v, 
     dim3 grid(num_splits, B * H);
     if (B * H > 65535) return ATTN_ERR_INVALID_ARG;   // grid.y limit
     cudaStream_t st = static_cast<cudaStream_t>(stream);
+    p.block_table = nullptr;
+    p.seq_lens = nullptr;
+    p.H = H;
+    p.page_shift = p.max_pages = p.num_pages = 0;
     if (d == 128)
-        attn_decode_partials_kernel<128><<<grid, DecodeTraits<128>::kThreads, 0, st>>>(p);
+        attn_decode_partials_kernel<128, false><<<grid, DecodeTraits<128>::kThreads, 0, st>>>(p);
     else
-        attn_decode_partials_kernel<64><<<grid, DecodeTraits<64>::kThreads, 0, st>>>(p);
+        attn_decode_partials_kernel<64, false><<<grid, DecodeTraits<64>::kThreads, 0, st>>>(p);
     return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+attn_status_t attn_decode_paged_partials(const void* q, const void* k_cache, const void* v_cache,
+                                         const int* block_table, const int* seq_lens,
+                                         float* o_part, float* lse_part, int B, int H, int d,
+                                         int page_size, int max_pages_per_seq, int num_pages,
+                                         float scale, int num_splits, void* stream) {
+    if (!q || !k_cache || !v_cache || !block_table || !seq_lens || !o_part || !lse_part)
+        return ATTN_ERR_INVALID_ARG;
+    if (!(scale > 0.f) || !std::isfinite(scale)) return ATTN_ERR_INVALID_ARG;
+    attn_status_t s = check_sizes(B, H, 1, 1);
+    if (s != ATTN_OK) return s;
+    if (num_splits < 1 || num_splits > 65535 || B * H > 65535) return ATTN_ERR_INVALID_ARG;
+    if (page_size < 16 || page_size > 1024 || (page_size & (page_size - 1)) != 0)
+        return ATTN_ERR_INVALID_ARG;
+    if (max_pages_per_seq < 1 || num_pages < 1) return ATTN_ERR_INVALID_ARG;
+    if ((long long)max_pages_per_seq * page_size > kMaxSeq) return ATTN_ERR_INVALID_ARG;
+    if ((long long)num_pages * H * page_size * d > (1ll << 46)) return ATTN_ERR_INVALID_ARG;
+    if (d != 64 && d != 128) return ATTN_ERR_UNSUPPORTED;
+    if (!aligned(q, 16) || !aligned(k_cache, 16) || !aligned(v_cache, 16) ||
+        !aligned(block_table, 4) || !aligned(seq_lens, 4) || !aligned(o_part, 4) ||
+        !aligned(lse_part, 4))
+        return ATTN_ERR_ALIGNMENT;
+    DecodeParams p;
+    p.q = static_cast<const uint16_t*>(q);
+    p.k = static_cast<const uint16_t*>(k_cache);
+    p.v = static_cast<const uint16_t*>(v_cache);
+    p.o_part = o_part;
+    p.lse_part = lse_part;
+    p.Nkv = 0;
+    p.L = 0;
+    p.S = num_splits;
+    p.scale_log2 = scale * kLog2e;
+    p.block_table = block_table;
+    p.seq_lens = seq_lens;
+    p.H = H;
+    p.page_shift = 0;
+    while ((1 << p.page_shift) < page_size) ++p.page_shift;
+    p.max_pages = max_pages_per_seq;
+    p.num_pages = num_pages;
+    dim3 grid(num_splits, B * H);
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (d == 128)
+        attn_decode_partials_kernel<128, true><<<grid, DecodeTraits<128>::kThreads, 0, st>>>(p);
+    else
+        attn_decode_partials_kernel<64, true><<<grid, DecodeTraits<64>::kThreads, 0, st>>>(p);
+    return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+attn_status_t attn_decode_paged(const void* q, const void* k_cache, const void* v_cache,
+                                const int* block_table, const int* seq_lens, void* o, float* lse,
+                                int B, int H, int d, int page_size, int max_pages_per_seq,
+                                int num_pages, float scale, int num_splits, void* workspace,
+                                size_t workspace_bytes, void* stream) {
+    if (!workspace || !o || !lse) return ATTN_ERR_INVALID_ARG;
+    const size_t need = attn_decode_workspace_bytes(B, H, d, num_splits);
+    if (need == 0) {
+        if (d != 64 && d != 128 && B >= 1 && H >= 1 && num_splits >= 1)
+            return ATTN_ERR_UNSUPPORTED;
+        return ATTN_ERR_INVALID_ARG;
+    }
+    if (workspace_bytes < need) return ATTN_ERR_INVALID_ARG;
+    if (!aligned(workspace, 256) || !aligned(o, 2) || !aligned(lse, 4)) return ATTN_ERR_ALIGNMENT;
+    float* o_part = static_cast<float*>(workspace);
+    const size_t o_bytes = ((size_t)B * H * num_splits * d * 4 + 255) / 256 * 256;
+    float* lse_part = reinterpret_cast<float*>(static_cast<char*>(workspace) + o_bytes);
+    attn_status_t s = attn_decode_paged_partials(q, k_cache, v_cache, block_table, seq_lens,
+                                                 o_part, lse_part, B, H, d, page_size,
+                                                 max_pages_per_seq, num_pages, scale, num_splits,
+                                                 stream);
+    if (s != ATTN_OK) return s;
+    return attn_lse_merge(o_part, lse_part, o, lse, B, H, num_splits, d, stream);
 }
 
 attn_status_t attn_lse_merge(const float* o_part, const float* lse_part, void* o, float* lse,
@@ -290,7 +368,9 @@ attn_status_t attn_status(void* stream) {
             return ATTN_ERR_CUDA;
     }
     if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
-    return (word & kDevErrTimeout) ? ATTN_ERR_TIMEOUT : ATTN_OK;
+    if (word & kDevErrTimeout) return ATTN_ERR_TIMEOUT;
+    if (word & kDevErrBadIndex) return ATTN_ERR_BAD_INDEX;
+    return ATTN_OK;
 }
 
 }  // extern "C"

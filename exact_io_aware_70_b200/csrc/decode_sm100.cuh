@@ -23,15 +23,23 @@ namespace eattn {
 
 struct DecodeParams {
     const uint16_t* q;   // bf16 [BH, D]
-    const uint16_t* k;   // bf16 [BH, Nkv, D]
-    const uint16_t* v;   // bf16 [BH, Nkv, D]
+    const uint16_t* k;   // bf16 [BH, Nkv, D]; paged: [num_pages, H, page_size, D]
+    const uint16_t* v;   // same layout as k
     float* o_part;       // fp32 [BH, S, D]
     float* lse_part;     // fp32 [BH, S]
-    int Nkv;
+    int Nkv;             // keys per row (contiguous layout)
     int S;               // number of chunks
-    int L;               // keys per chunk = ceil(Nkv / S)
+    int L;               // keys per chunk = ceil(Nkv / S) (contiguous layout)
     float scale_log2;    // scale * log2(e)
+    // paged layout only
+    const int* block_table;   // [B, max_pages]: physical page of each logical page
+    const int* seq_lens;      // [B]
+    int H, page_shift, max_pages, num_pages;
 };
+
+// Bit of the device status word: a block-table entry or sequence length was
+// out of range (the keys concerned were skipped, nothing out of range was read).
+constexpr unsigned kDevErrBadIndex = 2u;
 
 // 1: K/V loads of the decode kernel are marked evict-first in L2 (each byte is
 //    read exactly once). Measured: no gain for a prefill that follows, and
@@ -142,7 +150,9 @@ __device__ __forceinline__ int reduce_owner_index(int glane) {
                : ((glane >> 2) & 1) * 4 + ((glane >> 1) & 1) * 2 + (glane & 1);
 }
 
-template <int D>
+// PAGED: token j of sequence b is in physical page block_table[b][j >> page_shift],
+// slot j & (page_size - 1), of a cache laid out [num_pages][H][page_size][D].
+template <int D, bool PAGED>
 __global__ void __launch_bounds__(256)
     attn_decode_partials_kernel(const DecodeParams p) {
     using T = DecodeTraits<D>;
@@ -160,8 +170,19 @@ __global__ void __launch_bounds__(256)
     const int rs = tid / LPR;            // row slot within a pass
     const int glane = tid % LPR;         // lane within the row group
 
-    const long long j0 = (long long)c * p.L;
-    const long long j1 = min(j0 + (long long)p.L, (long long)p.Nkv);
+    int nkv = p.Nkv, L = p.L;
+    int b = 0, h = 0;
+    if (PAGED) {
+        b = bh / p.H;
+        h = bh - b * p.H;
+        const int len = p.seq_lens[b];
+        const int cap = p.max_pages << p.page_shift;
+        nkv = min(max(len, 0), cap);
+        if ((len < 0 || len > cap) && tid == 0 && c == 0) atomicOr(&g_attn_status, kDevErrBadIndex);
+        L = (nkv + p.S - 1) / p.S;
+    }
+    const long long j0 = (long long)c * L;
+    const long long j1 = min(j0 + (long long)L, (long long)nkv);
     const int n = j1 > j0 ? (int)(j1 - j0) : 0;
     float* o_out = p.o_part + ((size_t)bh * p.S + c) * D;
 
@@ -183,6 +204,22 @@ __global__ void __launch_bounds__(256)
     }
     const uint16_t* kbase = p.k + ((size_t)bh * p.Nkv + j0) * D + cc * 8;
     const uint16_t* vbase = p.v + ((size_t)bh * p.Nkv + j0) * D + cc * 8;
+    // Byte-free element offset of key j0 + i within K (and V); -1 if the key's page
+    // is out of range (then the key is skipped and the error is recorded).
+    const int* table = PAGED ? p.block_table + (size_t)b * p.max_pages : nullptr;
+    auto row_offset = [&](int i) -> long long {
+        if (!PAGED) return (long long)i * D;
+        const int j = (int)j0 + i;
+        const int page = __ldg(table + (j >> p.page_shift));
+        if (page < 0 || page >= p.num_pages) {
+            atomicOr(&g_attn_status, kDevErrBadIndex);
+            return -1;
+        }
+        return ((((long long)page * p.H + h) << p.page_shift) + (j & ((1 << p.page_shift) - 1))) *
+               D;
+    };
+    const uint16_t* kpaged = p.k + cc * 8;
+    const uint16_t* vpaged = p.v + cc * 8;
 
     const uint64_t pol = l2_policy_evict_first();
     float m_run = -INFINITY, l_run = 0.f;
@@ -195,21 +232,37 @@ __global__ void __launch_bounds__(256)
         // ---- scores for this sub-block: s_i = (scale*log2e) q . k_i
         for (int base = 0; base < SUB; base += RPP * NB) {
             uint4 kr[NB];
+            bool skip[NB];
 #pragma unroll
-            for (int b = 0; b < NB; ++b) {
-                const int i = base + rs + RPP * b;
-                kr[b] = i < nsub ? ld_stream_16B(kbase + (size_t)(sb + i) * D, pol)
-                                 : make_uint4(0, 0, 0, 0);
+            for (int r = 0; r < NB; ++r) {
+                const int i = base + rs + RPP * r;
+                skip[r] = i >= nsub;
+                if (PAGED && !skip[r]) {
+                    const long long off = row_offset(sb + i);
+                    skip[r] = off < 0;
+                    kr[r] = skip[r] ? make_uint4(0, 0, 0, 0) : ld_stream_16B(kpaged + off, pol);
+                } else {
+                    kr[r] = skip[r] ? make_uint4(0, 0, 0, 0)
+                                    : ld_stream_16B(kbase + (size_t)(sb + i) * D, pol);
+                }
             }
             float part[8];
 #pragma unroll
-            for (int b = 0; b < NB; ++b) part[b] = dot8(kr[b], qv);
+            for (int r = 0; r < NB; ++r) part[r] = dot8(kr[r], qv);
             const float sum = group_transpose_reduce8<LPR>(part, glane);
             const int owner = reduce_owner_index<D>(glane);
             const bool writer = (LPR == 16) ? ((glane & 1) == 0) : true;
             if (writer) {
                 const int i = base + rs + RPP * owner;
-                s_score[i] = i < nsub ? sum : -INFINITY;
+                bool skipped = i >= nsub;
+                if (PAGED) {
+                    // the owner's own slot tells whether its key was skipped
+                    // (lanes of one row group share rs, so skip[] agrees)
+#pragma unroll
+                    for (int r = 0; r < NB; ++r)
+                        if (r == owner) skipped = skip[r];
+                }
+                s_score[i] = skipped ? -INFINITY : sum;
             }
         }
         __syncthreads();
@@ -223,12 +276,16 @@ __global__ void __launch_bounds__(256)
         mx = s_red[0];
 #pragma unroll
         for (int w = 1; w < 8; ++w) mx = fmaxf(mx, s_red[w]);
-        const float m_new = fmaxf(m_run, mx);   // finite: the sub-block has >= 1 key
-        const float alpha = fast_exp2(m_run - m_new);   // 0 on the first sub-block
+        // m_new is finite unless every key so far was skipped (bad block-table
+        // entries); then nothing is accumulated and alpha stays 1.
+        const float m_new = fmaxf(m_run, mx);
+        const bool none = m_new == -INFINITY;
+        const float alpha = none ? 1.0f : fast_exp2(m_run - m_new);   // 0 on the first sub-block
+        const float base = none ? 0.0f : m_new;
         // ---- probabilities (unnormalised) and their sum
         float ls = 0.f;
         for (int i = tid; i < SUB; i += blockDim.x) {
-            const float e = fast_exp2(s_score[i] - m_new);
+            const float e = fast_exp2(s_score[i] - base);
             s_score[i] = e;
             ls += e;
         }
@@ -248,13 +305,20 @@ __global__ void __launch_bounds__(256)
         for (int base = 0; base < SUB; base += RPP * NB) {
             uint4 vr[NB];
 #pragma unroll
-            for (int b = 0; b < NB; ++b) {
-                const int i = base + rs + RPP * b;
-                vr[b] = i < nsub ? ld_stream_16B(vbase + (size_t)(sb + i) * D, pol)
-                                 : make_uint4(0, 0, 0, 0);
+            for (int r = 0; r < NB; ++r) {
+                const int i = base + rs + RPP * r;
+                bool skip_v = i >= nsub;
+                if (PAGED && !skip_v) {
+                    const long long off = row_offset(sb + i);
+                    skip_v = off < 0;
+                    vr[r] = skip_v ? make_uint4(0, 0, 0, 0) : ld_stream_16B(vpaged + off, pol);
+                } else {
+                    vr[r] = skip_v ? make_uint4(0, 0, 0, 0)
+                                   : ld_stream_16B(vbase + (size_t)(sb + i) * D, pol);
+                }
             }
 #pragma unroll
-            for (int b = 0; b < NB; ++b) axpy8(s_score[base + rs + RPP * b], vr[b], acc);
+            for (int r = 0; r < NB; ++r) axpy8(s_score[base + rs + RPP * r], vr[r], acc);
         }
         __syncthreads();                 // s_score and s_red are reused next sub-block
     }
@@ -262,7 +326,7 @@ __global__ void __launch_bounds__(256)
 #pragma unroll
     for (int i = 0; i < 8; ++i) s_acc[rs][cc * 8 + i] = acc[i];
     __syncthreads();
-    const float inv = 1.0f / l_run;
+    const float inv = l_run > 0.f ? 1.0f / l_run : 0.f;   // l_run = 0: every key skipped
     for (int x = tid; x < D; x += blockDim.x) {
         float s = 0.f;
 #pragma unroll 4
@@ -270,7 +334,8 @@ __global__ void __launch_bounds__(256)
         o_out[x] = s * inv;
     }
     if (tid == 0)
-        p.lse_part[(size_t)bh * p.S + c] = (m_run + log2f(l_run)) * 0.69314718055994531f;
+        p.lse_part[(size_t)bh * p.S + c] =
+            l_run > 0.f ? (m_run + log2f(l_run)) * 0.69314718055994531f : -INFINITY;
 }
 
 // ------------------------------------------------------------------ merge --

@@ -49,7 +49,8 @@ typedef enum {
     ATTN_ERR_ALIGNMENT = 3,
     ATTN_ERR_CUDA = 4,
     ATTN_ERR_TIMEOUT = 5,
-    ATTN_ERR_SCRATCH_LIMIT = 6
+    ATTN_ERR_SCRATCH_LIMIT = 6,
+    ATTN_ERR_BAD_INDEX = 7
 } attn_status_t;
 
 /* Version of this ABI (bumped on any incompatible change). */
@@ -134,6 +135,45 @@ attn_status_t attn_decode_splitkv(const void *q, const void *k, const void *v, v
                                   float *lse, int B, int H, int Nkv, int d, float scale,
                                   int num_splits, void *workspace, size_t workspace_bytes,
                                   void *stream);
+
+/*
+ * Paged-KV split-KV decode, step 1: per-chunk partials over a paged KV cache.
+ *
+ * Defines: the "paged variants for decode" the serving systems use
+ * (mantramindai, "Versions", last paragraph; PagedAttention in appliedaiprep,
+ * "What interviewers probe next"). The pages give no layout; this library's:
+ * the cache holds num_pages physical pages of page_size tokens for every head,
+ *   k_cache, v_cache  bf16 [num_pages, H, page_size, d]   (read)
+ * token j of sequence b is in physical page block_table[b][j / page_size],
+ * slot j % page_size;
+ *   block_table  int32 [B, max_pages_per_seq]           (read)
+ *   seq_lens     int32 [B], tokens cached per sequence   (read)
+ *   q            bf16 [B, H, 1, d]                       (read)
+ *   o_part, lse_part as for attn_decode_partials, with chunks of
+ *   ceil(seq_lens[b] / num_splits) tokens per sequence.
+ * page_size is a power of two in [16, 1024]. A sequence of length 0 yields
+ * empty chunks (O = 0, LSE = -inf after the merge). Table entries outside
+ * [0, num_pages) and lengths outside [0, max_pages_per_seq * page_size] are
+ * never dereferenced: the keys concerned are skipped and attn_status()
+ * reports ATTN_ERR_BAD_INDEX.
+ */
+attn_status_t attn_decode_paged_partials(const void *q, const void *k_cache, const void *v_cache,
+                                         const int *block_table, const int *seq_lens,
+                                         float *o_part, float *lse_part, int B, int H, int d,
+                                         int page_size, int max_pages_per_seq, int num_pages,
+                                         float scale, int num_splits, void *stream);
+
+/*
+ * Paged-KV split-KV decode, both steps: attn_decode_paged_partials into
+ * `workspace` (attn_decode_workspace_bytes(B, H, d, num_splits) bytes, 256-byte
+ * aligned, caller-owned), then attn_lse_merge into o [B, H, 1, d] (bf16) and
+ * lse [B, H, 1] (fp32).
+ */
+attn_status_t attn_decode_paged(const void *q, const void *k_cache, const void *v_cache,
+                                const int *block_table, const int *seq_lens, void *o, float *lse,
+                                int B, int H, int d, int page_size, int max_pages_per_seq,
+                                int num_pages, float scale, int num_splits, void *workspace,
+                                size_t workspace_bytes, void *stream);
 
 /*
  * Split-KV decode for callers that cannot allocate device memory.

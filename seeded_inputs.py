@@ -57,6 +57,11 @@ WORKLOADS = {
     "decode_32k": Workload("decode_32k", 16, 32, 1, 32768, 128, False, 4, num_splits=64),
 }
 
+# The paged variant of decode_32k: the same 16 x 32 rows over 32768 cached tokens,
+# stored in 256-token pages placed in a random physical order.
+PAGED_DECODE = dict(name="decode_32k_paged", B=16, H=32, seq_len=32768, d=128, page_size=256,
+                    num_splits=64, seed=5)
+
 
 def make_qkv(B: int, H: int, Nq: int, Nkv: int, d: int, seed: int,
              device: str = "cpu"):
@@ -88,6 +93,28 @@ def make_partials(B: int, H: int, S: int, d: int, seed: int, empty_every: int = 
         lse[..., ::empty_every] = float("-inf")
         o[..., ::empty_every, :] = 0.0
     return o, lse
+
+
+def make_paged_cache(B: int, H: int, seq_lens, d: int, page_size: int, seed: int,
+                     device: str = "cpu", spare_pages: int = 3):
+    """A paged KV cache for decode: q [B,H,1,d] and K, V caches
+    [num_pages, H, page_size, d], all bf16 i.i.d. N(0,1) (drawn q, K, V), with a
+    block table [B, max_pages] int32 that assigns each sequence's logical pages
+    to physical pages in a seeded random order, and seq_lens [B] int32.
+    Unused table entries point at spare pages; spare pages hold data too."""
+    g = torch.Generator(device="cpu")
+    g.manual_seed(seed)
+    lens = [int(x) for x in seq_lens]
+    max_pages = max(1, max((n + page_size - 1) // page_size for n in lens))
+    num_pages = B * max_pages + spare_pages
+    perm = torch.randperm(num_pages, generator=g)
+    table = perm[:B * max_pages].reshape(B, max_pages).to(torch.int32)
+    gd = torch.Generator(device=device)
+    gd.manual_seed(seed)
+    q = torch.randn((B, H, 1, d), generator=gd, device=device).to(torch.bfloat16)
+    k = torch.randn((num_pages, H, page_size, d), generator=gd, device=device).to(torch.bfloat16)
+    v = torch.randn((num_pages, H, page_size, d), generator=gd, device=device).to(torch.bfloat16)
+    return q, k, v, table.to(device), torch.tensor(lens, dtype=torch.int32, device=device)
 
 
 def bf16_bits(t: torch.Tensor):

@@ -33,7 +33,7 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
-from seeded_inputs import WORKLOADS, make_workload  # noqa: E402
+from seeded_inputs import WORKLOADS, make_qkv, make_workload  # noqa: E402
 
 METRIC = "attn fwd TFLOP/s & % BF16 tensor peak; decode KV GB/s & % HBM peak"
 PREFILL = WORKLOADS["prefill_8k"]
@@ -243,6 +243,82 @@ def cpu_baseline(budget_s=8.0):
                    f"({dc['bytes'] / 1e9:.2f} GB of K/V in {dc['seconds']:.2f} s)"),
         "decode": {"value": dc["bytes"] / dc["seconds"] / 1e9, "unit": "GB/s"},
     }
+
+
+def naive_comparison(dev, flash_ms_8k):
+    """The naive three-step attention the pages contrast with (S = scale QK^T and
+    P = softmax(S) written to HBM in bf16, then O = PV), run with torch on the
+    same GPU: its time on prefill_8k against this library's, its accuracy on
+    sampled rows against the oracle, and the device memory each needs at 2K,
+    4K and 8K tokens (the pages' "10x less memory at 2K, 20x at 4K" claim).
+    A comparison only: nothing of it is on the library's path."""
+    import numpy as np
+    import torch
+
+    import exact_io_aware_70_b200 as ea
+    w = PREFILL
+
+    def naive(q, k, v):
+        s_ = torch.matmul(q, k.transpose(-1, -2)) * w.scale       # S materialised (bf16)
+        n = q.shape[2]
+        s_.masked_fill_(torch.ones(n, n, dtype=torch.bool, device=dev).triu(1), float("-inf"))
+        p_ = torch.softmax(s_, dim=-1)                              # P materialised (bf16)
+        del s_
+        return torch.matmul(p_, v)
+
+    out = {"what": "torch bf16 matmul -> masked softmax -> matmul, S and P materialised"}
+    q, k, v = make_workload(w, device="cuda")
+    for _ in range(2):
+        naive(q, k, v)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    reps = 5
+    for _ in range(reps):
+        o_n = naive(q, k, v)
+    e1.record()
+    torch.cuda.synchronize()
+    naive_ms = e0.elapsed_time(e1) / reps
+    out.update(workload="prefill_8k", naive_ms=naive_ms, flash_ms=flash_ms_8k,
+               speedup=naive_ms / flash_ms_8k,
+               score_matrix_bytes_per_head=w.Nq * w.Nkv * 2,
+               score_matrix_bytes_total=w.B * w.H * w.Nq * w.Nkv * 2)
+    # accuracy of the naive bf16 path on sampled rows of head 0 (oracle = fp64 definition)
+    try:
+        import oracle
+        from seeded_inputs import bf16_bits
+        rows = np.linspace(0, w.Nq - 1, 64).astype(np.int64)
+        ro, _ = oracle.get().attn_rows_bf16(bf16_bits(q[0, 0].cpu()), bf16_bits(k[0, 0].cpu()),
+                                            bf16_bits(v[0, 0].cpu()), rows, w.causal, w.scale)
+        out["naive_max_abs_err_O_sampled"] = float(np.abs(o_n[0, 0, rows].float().cpu().numpy()
+                                                          - ro).max())
+    except Exception as exc:   # the comparison is informational
+        out["naive_accuracy"] = f"not measured: {exc}"
+    del q, k, v, o_n
+    # peak device memory above the inputs, naive vs this library
+    mem = {}
+    for n in (2048, 4096, 8192):
+        qn, kn, vn = make_qkv(1, w.H, n, n, w.d, 7, device="cuda")
+        torch.cuda.synchronize()
+        torch.cuda.reset_peak_memory_stats()
+        base = torch.cuda.memory_allocated()
+        o_ = naive(qn, kn, vn)
+        torch.cuda.synchronize()
+        naive_extra = torch.cuda.max_memory_allocated() - base
+        del o_
+        torch.cuda.synchronize()
+        torch.cuda.reset_peak_memory_stats()
+        base = torch.cuda.memory_allocated()
+        of = torch.empty_like(qn)
+        lf = torch.empty((1, w.H, n), dtype=torch.float32, device=dev)
+        ea.attn_fwd(qn, kn, vn, of, lf, True, w.scale)
+        torch.cuda.synchronize()
+        flash_extra = torch.cuda.max_memory_allocated() - base
+        mem[str(n)] = {"naive_bytes": int(naive_extra), "flash_bytes": int(flash_extra),
+                       "ratio": naive_extra / flash_extra}
+        del qn, kn, vn, of, lf
+    out["memory_above_inputs_H32_d128"] = mem
+    return out
 
 
 def run_reference(args):
@@ -548,6 +624,8 @@ def run_ours(args):
     })
     if ws == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(args.cpu_budget)
+    if ws == 1 and pw is PREFILL and not args.no_naive:
+        line["naive_comparison"] = naive_comparison(dev, kms["attn_fwd_sm100"])
     print(json.dumps(line), flush=True)
     return 0
 
@@ -566,6 +644,8 @@ def main():
                     help="override the batch size (small profiling captures only)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-naive", action="store_true",
+                    help="skip the naive materialising attention comparison")
     ap.add_argument("--cpu-budget", type=float, default=8.0,
                     help="seconds of oracle work for the CPU baseline")
     args = ap.parse_args()

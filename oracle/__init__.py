@@ -50,6 +50,11 @@ class Oracle:
         lib.oracle_decode_paged_bf16.argtypes = [_u16p, _u16p, _u16p, _i32p, _i32p, _c_long,
                                                  _c_long, _c_long, _c_long, _c_long, _c_long,
                                                  ctypes.c_double, _dp, _dp]
+        lib.oracle_attn_bwd_head_f64.argtypes = [_dp, _dp, _dp, _dp, _c_long, _c_long, _c_long,
+                                                 ctypes.c_int, ctypes.c_double, _dp, _dp, _dp]
+        lib.oracle_attn_bwd_bf16.argtypes = [_u16p, _u16p, _u16p, _u16p, _c_long, _c_long,
+                                             _c_long, _c_long, _c_long, ctypes.c_int,
+                                             ctypes.c_double, _dp, _dp, _dp]
         lib.oracle_num_threads.restype = ctypes.c_int
         lib.oracle_set_num_threads.argtypes = [ctypes.c_int]
         self.lib = lib
@@ -114,6 +119,35 @@ class Oracle:
         if rc:
             raise RuntimeError("oracle_decode_partials_bf16 failed")
         return o, lse
+
+    def attn_bwd_head_f64(self, q, k, v, dout, causal: bool, scale: float):
+        """Gradients of sum(dout * O) for one head -> (dq, dk, dv) in double."""
+        q, k, v, dout = (np.ascontiguousarray(x, dtype=np.float64) for x in (q, k, v, dout))
+        Nq, d = q.shape
+        Nkv = k.shape[0]
+        dq, dk, dv = np.zeros((Nq, d)), np.zeros((Nkv, d)), np.zeros((Nkv, d))
+        rc = self.lib.oracle_attn_bwd_head_f64(_ptr(q, _dp), _ptr(k, _dp), _ptr(v, _dp),
+                                               _ptr(dout, _dp), Nq, Nkv, d, int(causal),
+                                               float(scale), _ptr(dq, _dp), _ptr(dk, _dp),
+                                               _ptr(dv, _dp))
+        if rc:
+            raise RuntimeError("oracle_attn_bwd_head_f64 failed")
+        return dq, dk, dv
+
+    def attn_bwd_bf16(self, q_bits, k_bits, v_bits, dout_bits, causal: bool, scale: float):
+        """[B,H,N,d] uint16 inputs -> (dq, dk, dv) double arrays of the same shapes."""
+        B, H, Nq, d = q_bits.shape
+        Nkv = k_bits.shape[2]
+        q, k, v, do = (np.ascontiguousarray(x, dtype=np.uint16)
+                       for x in (q_bits, k_bits, v_bits, dout_bits))
+        dq, dk, dv = np.zeros((B, H, Nq, d)), np.zeros((B, H, Nkv, d)), np.zeros((B, H, Nkv, d))
+        rc = self.lib.oracle_attn_bwd_bf16(_ptr(q, _u16p), _ptr(k, _u16p), _ptr(v, _u16p),
+                                           _ptr(do, _u16p), B, H, Nq, Nkv, d, int(causal),
+                                           float(scale), _ptr(dq, _dp), _ptr(dk, _dp),
+                                           _ptr(dv, _dp))
+        if rc:
+            raise RuntimeError("oracle_attn_bwd_bf16 failed")
+        return dq, dk, dv
 
     def decode_paged_bf16(self, q_bits, k_cache_bits, v_cache_bits, block_table, seq_lens,
                           scale: float):
@@ -182,7 +216,7 @@ def get() -> Oracle:
 
 
 def build_mutant(n: int, out_dir: str) -> Oracle:
-    """A copy of the oracle with planted mistake ``n`` (1..11), for the pin tests."""
+    """A copy of the oracle with planted mistake ``n`` (1..13), for the pin tests."""
     out = os.path.join(out_dir, f"liboracle_mutant{n}.so")
     _build.build(out=out, mutant=n, force=True)
     return Oracle(out)

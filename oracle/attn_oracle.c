@@ -397,6 +397,99 @@ int oracle_decode_paged_bf16(const uint16_t *q, const uint16_t *k_cache, const u
     return 0;
 }
 
+/*
+ * Backward pass: gradients of L = sum(dO * O) for one head, the gradients the
+ * pages say FlashAttention recomputes from Q, K and V instead of storing P
+ * ("Describe Flash Attention at a high level" (mantramindai), "The two ideas",
+ * item 3, and "Follow-up questions to expect": outputs and gradients match
+ * standard attention; "How FlashAttention Speeds Up the Attention Layer"
+ * (hassanahmed.net), the backward-pass paragraph). The pages print no
+ * formulas; these are the chain rule applied to the definition above, with S
+ * and P materialised:
+ *   dV = P^T dO;  dP = dO V^T;  D_i = sum_j P_ij dP_ij (= sum_c dO_ic O_ic);
+ *   dS = P o (dP - D);  dQ = scale dS K;  dK = scale dS^T Q.
+ *   q, dq [Nq, d]; k, v, dk, dv [Nkv, d]; dout [Nq, d].
+ */
+int oracle_attn_bwd_head_f64(const double *q, const double *k, const double *v,
+                             const double *dout, long Nq, long Nkv, long d, int causal,
+                             double scale, double *dq, double *dk, double *dv) {
+    if (Nq < 0 || Nkv < 0 || d <= 0) return -1;
+    size_t nn = (size_t)(Nq > 0 ? Nq : 1) * (size_t)(Nkv > 0 ? Nkv : 1);
+    double *P = (double *)malloc(nn * sizeof(double));
+    double *dS = (double *)malloc(nn * sizeof(double));
+    if (!P || !dS) { free(P); free(dS); return -1; }
+    /* recompute S and P */
+#pragma omp parallel for schedule(dynamic, 4)
+    for (long i = 0; i < Nq; ++i) {
+        score_row(q + i * d, k, Nkv, d, i, Nq, causal, scale, P + i * Nkv);
+        softmax_row(P + i * Nkv, Nkv);
+    }
+    /* dP, D and dS, row by row */
+#pragma omp parallel for schedule(dynamic, 4)
+    for (long i = 0; i < Nq; ++i) {
+        double D = 0.0;
+        for (long j = 0; j < Nkv; ++j) {
+            double dp = 0.0;
+            for (long c = 0; c < d; ++c) dp += dout[i * d + c] * v[j * d + c];
+            dS[i * Nkv + j] = dp;
+            D += P[i * Nkv + j] * dp;
+        }
+        for (long j = 0; j < Nkv; ++j) {
+#if ORACLE_MUTANT == 12 /* dropped the D term */
+            dS[i * Nkv + j] = P[i * Nkv + j] * dS[i * Nkv + j];
+#else
+            dS[i * Nkv + j] = P[i * Nkv + j] * (dS[i * Nkv + j] - D);
+#endif
+        }
+    }
+    /* dQ = scale dS K */
+#pragma omp parallel for schedule(static)
+    for (long i = 0; i < Nq; ++i)
+        for (long c = 0; c < d; ++c) {
+            double acc = 0.0;
+            for (long j = 0; j < Nkv; ++j) acc += dS[i * Nkv + j] * k[j * d + c];
+            dq[i * d + c] = scale * acc;
+        }
+    /* dK = scale dS^T Q, dV = P^T dO */
+#pragma omp parallel for schedule(static)
+    for (long j = 0; j < Nkv; ++j)
+        for (long c = 0; c < d; ++c) {
+            double ak = 0.0, av = 0.0;
+            for (long i = 0; i < Nq; ++i) {
+                ak += dS[i * Nkv + j] * q[i * d + c];
+                av += P[i * Nkv + j] * dout[i * d + c];
+            }
+#if ORACLE_MUTANT == 13 /* dK without the scale */
+            dk[j * d + c] = ak;
+#else
+            dk[j * d + c] = scale * ak;
+#endif
+            dv[j * d + c] = av;
+        }
+    free(P); free(dS);
+    return 0;
+}
+
+/* Backward on bf16 inputs [B, H, N, d]; dq [B,H,Nq,d], dk and dv [B,H,Nkv,d] double. */
+int oracle_attn_bwd_bf16(const uint16_t *q, const uint16_t *k, const uint16_t *v,
+                         const uint16_t *dout, long B, long H, long Nq, long Nkv, long d,
+                         int causal, double scale, double *dq, double *dk, double *dv) {
+    if (B < 0 || H < 0 || Nq < 0 || Nkv < 0 || d <= 0) return -1;
+    for (long bh = 0; bh < B * H; ++bh) {
+        double *qh = widen_bf16(q + bh * Nq * d, (size_t)(Nq * d));
+        double *kh = widen_bf16(k + bh * Nkv * d, (size_t)(Nkv * d));
+        double *vh = widen_bf16(v + bh * Nkv * d, (size_t)(Nkv * d));
+        double *oh = widen_bf16(dout + bh * Nq * d, (size_t)(Nq * d));
+        int rc = (qh && kh && vh && oh) ? 0 : -1;
+        if (rc == 0)
+            rc = oracle_attn_bwd_head_f64(qh, kh, vh, oh, Nq, Nkv, d, causal, scale,
+                                          dq + bh * Nq * d, dk + bh * Nkv * d, dv + bh * Nkv * d);
+        free(qh); free(kh); free(vh); free(oh);
+        if (rc) return rc;
+    }
+    return 0;
+}
+
 /* number of OpenMP threads the oracle will use (1 without OpenMP) */
 int oracle_num_threads(void) {
 #ifdef _OPENMP

@@ -362,10 +362,65 @@ def pin_paged_golden(orc):
     assert lse[1, 0] == -math.inf
 
 
+# ---------------------------------------------------------------------------
+# 8. Backward pass (gradients of sum(dO * O))
+# ---------------------------------------------------------------------------
+def pin_bwd_torch_autograd(orc):
+    """torch autograd through scaled_dot_product_attention in float64 (CPU)."""
+    F = torch.nn.functional
+    for causal, (Nq, Nkv, d) in ((False, (7, 11, 8)), (True, (12, 12, 4)), (False, (1, 30, 16))):
+        q, k, v, do = (_rand(s_, 40 + i) for i, s_ in enumerate(((Nq, d), (Nkv, d), (Nkv, d),
+                                                                  (Nq, d))))
+        scale = 1.0 / math.sqrt(d)
+        dq, dk, dv = orc.attn_bwd_head_f64(q, k, v, do, causal, scale)
+        tq, tk, tv = (torch.from_numpy(x)[None, None].requires_grad_(True) for x in (q, k, v))
+        out = F.scaled_dot_product_attention(tq, tk, tv, is_causal=causal, scale=scale)
+        out.backward(torch.from_numpy(do)[None, None])
+        _close(dq, tq.grad[0, 0].numpy(), 1e-10, "autograd dQ")
+        _close(dk, tk.grad[0, 0].numpy(), 1e-10, "autograd dK")
+        _close(dv, tv.grad[0, 0].numpy(), 1e-10, "autograd dV")
+
+
+def pin_bwd_finite_differences(orc):
+    """Central differences of L = sum(dO * O) through the forward oracle."""
+    Nq, Nkv, d, scale = 5, 6, 3, 0.7
+    q, k, v, do = _rand((Nq, d), 50), _rand((Nkv, d), 51), _rand((Nkv, d), 52), _rand((Nq, d), 53)
+    for causal in (False, True):
+        dq, dk, dv = orc.attn_bwd_head_f64(q, k, v, do, causal, scale)
+
+        def loss(q_, k_, v_):
+            o, _ = orc.attn_head_f64(q_, k_, v_, causal, scale)
+            return float((o * do).sum())
+        h = 1e-6
+        for name, x, g in (("q", q, dq), ("k", k, dk), ("v", v, dv)):
+            for (a, b) in ((0, 0), (x.shape[0] - 1, d - 1), (2, 1)):
+                xp, xm = x.copy(), x.copy()
+                xp[a, b] += h
+                xm[a, b] -= h
+                args_p = {"q": (xp, k, v), "k": (q, xp, v), "v": (q, k, xp)}[name]
+                args_m = {"q": (xm, k, v), "k": (q, xm, v), "v": (q, k, xm)}[name]
+                num = (loss(*args_p) - loss(*args_m)) / (2 * h)
+                _close(g[a, b], num, 1e-6, f"finite difference d{name}[{a},{b}] causal{causal}")
+
+
+def pin_bwd_invariants(orc):
+    """Softmax is unchanged by adding one vector to every key, so the key
+    gradients sum to zero; with q = 0 the weights are uniform, so dV_j is the
+    mean of dO over the rows (non-causal)."""
+    Nq, Nkv, d = 6, 9, 4
+    q, k, v, do = _rand((Nq, d), 54), _rand((Nkv, d), 55), _rand((Nkv, d), 56), _rand((Nq, d), 57)
+    for causal in (False, True):
+        _, dk, _ = orc.attn_bwd_head_f64(q, k, v, do, causal, 0.5)
+        _close(dk.sum(axis=0), np.zeros(d), 1e-12, "sum of dK")
+    _, _, dv = orc.attn_bwd_head_f64(np.zeros((Nq, d)), k, v, do, False, 0.5)
+    _close(dv, np.tile(do.sum(axis=0) / Nkv, (Nkv, 1)), 1e-12, "uniform weights dV")
+
+
 ALL_PINS = [
     pin_worked_example, pin_golden_cases, pin_probabilities, pin_constant_values,
     pin_identical_keys, pin_zero_query, pin_causal_first_row, pin_key_permutation,
     pin_value_linearity, pin_causal_is_truncation, pin_torch_sdpa, pin_merge_any_chunking,
     pin_partials_are_chunk_attention, pin_merge_batched_matches_single, pin_bf16_entry,
     pin_paged_matches_contiguous, pin_paged_golden,
+    pin_bwd_torch_autograd, pin_bwd_finite_differences, pin_bwd_invariants,
 ]

@@ -24,6 +24,8 @@ MUTANTS = {
     9: "merge weights not normalised",
     10: "paged decode ignores the block table",
     11: "paged decode reads one token past the sequence",
+    12: "backward drops the D term",
+    13: "backward dK without the scale",
 }
 
 

@@ -57,6 +57,10 @@ lib.attn_decode_paged_partials.restype = _i
 lib.attn_decode_paged_partials.argtypes = [_vp] * 7 + [_i] * 6 + [_f, _i, _vp]
 lib.attn_decode_paged.restype = _i
 lib.attn_decode_paged.argtypes = [_vp] * 7 + [_i] * 6 + [_f, _i, _vp, _sz, _vp]
+lib.attn_bwd_workspace_bytes.restype = _sz
+lib.attn_bwd_workspace_bytes.argtypes = [_i, _i, _i, _i]
+lib.attn_bwd.restype = _i
+lib.attn_bwd.argtypes = [_vp] * 9 + [_i] * 6 + [_f, _vp, _sz, _vp]
 lib.attn_status.restype = _i
 lib.attn_status.argtypes = [_vp]
 
@@ -186,6 +190,32 @@ def attn_decode_paged(q, k_cache, v_cache, block_table, seq_lens, o, lse, scale:
                                  P if num_pages is None else int(num_pages), float(scale),
                                  int(num_splits), _tensor(workspace, torch.uint8, "workspace"),
                                  workspace.numel(), _stream(stream)), "attn_decode_paged")
+
+
+def attn_bwd_workspace_bytes(B: int, H: int, Nq: int, d: int) -> int:
+    return int(lib.attn_bwd_workspace_bytes(B, H, Nq, d))
+
+
+def attn_bwd(q, k, v, o, dout, lse, dq, dk, dv, causal: bool, scale: float, workspace,
+             stream=None) -> None:
+    """dQ, dK, dV of sum(dO*O). q/o/dout/dq [B,H,Nq,d], k/v/dk/dv [B,H,Nkv,d] bf16; lse [B,H,Nq] fp32;
+    workspace: a device buffer of at least attn_bwd_workspace_bytes(B, H, Nq, d) bytes."""
+    import torch
+    B, H, Nq, d = q.shape
+    Nkv = k.shape[2]
+    qs, ks = (B, H, Nq, d), (B, H, Nkv, d)
+    if any(tuple(t.shape) != qs for t in (o, dout, dq)) \
+            or any(tuple(t.shape) != ks for t in (k, v, dk, dv)) or tuple(lse.shape) != (B, H, Nq):
+        raise ValueError("attn_bwd: inconsistent shapes")
+    if not workspace.is_contiguous():
+        raise ValueError("attn_bwd: workspace must be contiguous")
+    _check(lib.attn_bwd(_tensor(q, torch.bfloat16, "q"), _tensor(k, torch.bfloat16, "k"),
+                        _tensor(v, torch.bfloat16, "v"), _tensor(o, torch.bfloat16, "o"),
+                        _tensor(dout, torch.bfloat16, "dout"), _tensor(lse, torch.float32, "lse"),
+                        _tensor(dq, torch.bfloat16, "dq"), _tensor(dk, torch.bfloat16, "dk"),
+                        _tensor(dv, torch.bfloat16, "dv"), B, H, Nq, Nkv, d, int(bool(causal)),
+                        float(scale), ctypes.c_void_p(workspace.data_ptr()),
+                        workspace.numel() * workspace.element_size(), _stream(stream)), "attn_bwd")
 
 
 def attn_status(stream=None) -> int:

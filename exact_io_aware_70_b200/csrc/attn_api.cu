@@ -18,6 +18,7 @@ namespace eattn {
 __device__ unsigned g_attn_status = 0;
 }  // namespace eattn
 
+#include "bwd_sm100.cuh"
 #include "decode_sm100.cuh"
 #include "fwd_sm100.cuh"
 
@@ -86,6 +87,7 @@ bool encode_bf16_map(CUtensorMap* map, const void* base, int BH, int N, int D) {
 struct DeviceInfo {
     int sms = 0;
     bool fwd_attr_set[4] = {false, false, false, false};
+    bool bwd_attr_set[4] = {false, false, false, false};
 };
 DeviceInfo g_dev[64];
 std::mutex g_dev_mu;
@@ -121,6 +123,37 @@ attn_status_t launch_fwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUt
     }
     const int grid = p.num_units < sms ? p.num_units : sms;
     kern<<<grid, T::kThreads, T::kSmemBytes, stream>>>(tq, tk, tv, p);
+    return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+template <int D, bool CAUSAL>
+attn_status_t launch_bwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                         const CUtensorMap& tdo, const BwdParams& p, cudaStream_t stream) {
+    using T = BwdTraits<D>;
+    const int dev = current_device();
+    if (dev < 0 || dev >= 64) return ATTN_ERR_CUDA;
+    auto kern = attn_bwd_sm100_kernel<D, CAUSAL>;
+    {
+        std::lock_guard<std::mutex> lk(g_dev_mu);
+        DeviceInfo& di = g_dev[dev];
+        const int slot = (D == 128 ? 2 : 0) + (CAUSAL ? 1 : 0);
+        if (!di.bwd_attr_set[slot]) {
+            if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     T::kSmemBytes) != cudaSuccess)
+                return ATTN_ERR_CUDA;
+            di.bwd_attr_set[slot] = true;
+        }
+    }
+    const long long rows = (long long)p.BH * p.Nq;
+    constexpr int kRowsPerBlock = 256 / (D / 8);
+    attn_bwd_preprocess_kernel<D>
+        <<<(unsigned)((rows + kRowsPerBlock - 1) / kRowsPerBlock), 256, 0, stream>>>(p);
+    // key blocks along x so that the CTAs resident at one time share a few
+    // heads' Q and dO tiles in L2
+    dim3 grid((p.Nkv + 127) / 128, p.BH);
+    kern<<<grid, T::kThreads, T::kSmemBytes, stream>>>(tq, tk, tv, tdo, p);
+    attn_bwd_postprocess_kernel<D>
+        <<<(unsigned)((rows * D / 8 + 255) / 256), 256, 0, stream>>>(p);
     return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
 
@@ -347,6 +380,58 @@ attn_status_t attn_decode_splitkv(const void* q, const void* k, const void* v, v
                                            num_splits, stream);
     if (s != ATTN_OK) return s;
     return attn_lse_merge(o_part, lse_part, o, lse, B, H, num_splits, d, stream);
+}
+
+size_t attn_bwd_workspace_bytes(int B, int H, int Nq, int d) {
+    if (B < 1 || H < 1 || Nq < 1 || (d != 64 && d != 128)) return 0;
+    const size_t rows = (size_t)B * H * Nq;
+    return (rows * 4 + 255) / 256 * 256 + rows * d * 4;
+}
+
+attn_status_t attn_bwd(const void* q, const void* k, const void* v, const void* o,
+                       const void* dout, const float* lse, void* dq, void* dk, void* dv, int B,
+                       int H, int Nq, int Nkv, int d, int causal, float scale, void* workspace,
+                       size_t workspace_bytes, void* stream) {
+    if (!q || !k || !v || !o || !dout || !lse || !dq || !dk || !dv || !workspace)
+        return ATTN_ERR_INVALID_ARG;
+    if (causal != 0 && causal != 1) return ATTN_ERR_INVALID_ARG;
+    if (!(scale > 0.f) || !std::isfinite(scale)) return ATTN_ERR_INVALID_ARG;
+    attn_status_t s = check_sizes(B, H, Nq, Nkv);
+    if (s != ATTN_OK) return s;
+    if (d != 64 && d != 128) return ATTN_ERR_UNSUPPORTED;
+    const int BH = B * H;
+    if (BH > 65535) return ATTN_ERR_INVALID_ARG;   // grid.y limit
+    if ((long long)BH * Nq * d / 2048 >= (1ll << 31)) return ATTN_ERR_INVALID_ARG;
+    if (workspace_bytes < attn_bwd_workspace_bytes(B, H, Nq, d)) return ATTN_ERR_INVALID_ARG;
+    if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) ||
+        !aligned(dout, 16) || !aligned(dq, 16) || !aligned(dk, 16) || !aligned(dv, 16) ||
+        !aligned(lse, 4) || !aligned(workspace, 256))
+        return ATTN_ERR_ALIGNMENT;
+    CUtensorMap tq, tk, tv, tdo;
+    if (!encode_bf16_map(&tq, q, BH, Nq, d) || !encode_bf16_map(&tk, k, BH, Nkv, d) ||
+        !encode_bf16_map(&tv, v, BH, Nkv, d) || !encode_bf16_map(&tdo, dout, BH, Nq, d))
+        return ATTN_ERR_CUDA;
+    const size_t rows = (size_t)BH * Nq;
+    BwdParams p;
+    p.o = static_cast<const uint16_t*>(o);
+    p.dout = static_cast<const uint16_t*>(dout);
+    p.lse = lse;
+    p.delta = static_cast<float*>(workspace);
+    p.dq_acc = reinterpret_cast<float*>(static_cast<char*>(workspace) + (rows * 4 + 255) / 256 * 256);
+    p.dq = static_cast<uint16_t*>(dq);
+    p.dk = static_cast<uint16_t*>(dk);
+    p.dv = static_cast<uint16_t*>(dv);
+    p.BH = BH;
+    p.Nq = Nq;
+    p.Nkv = Nkv;
+    p.scale = scale;
+    p.scale_log2 = scale * kLog2e;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (d == 128)
+        return causal ? launch_bwd<128, true>(tq, tk, tv, tdo, p, st)
+                      : launch_bwd<128, false>(tq, tk, tv, tdo, p, st);
+    return causal ? launch_bwd<64, true>(tq, tk, tv, tdo, p, st)
+                  : launch_bwd<64, false>(tq, tk, tv, tdo, p, st);
 }
 
 attn_status_t attn_selftest_wait_timeout(unsigned limit_us, void* stream) {

@@ -199,6 +199,47 @@ attn_status_t attn_decode_splitkv_noalloc(const void *q, const void *k, const vo
                                           int num_splits, void *stream);
 
 /*
+ * Backward pass: bytes of device workspace attn_bwd needs, or 0 if the
+ * arguments are invalid. Layout (owned by the caller, 256-byte aligned):
+ * fp32 D [B, H, Nq] padded to 256 bytes, then the fp32 dQ accumulator
+ * [B, H, Nq, d]. Nothing in it needs initialising.
+ */
+size_t attn_bwd_workspace_bytes(int B, int H, int Nq, int d);
+
+/*
+ * Backward pass: dQ, dK, dV of L = sum(dO * O) for the attention attn_fwd
+ * computes, recomputing the score and probability tiles from Q, K and the
+ * forward pass's LSE instead of storing P.
+ *
+ * Defines: "Describe Flash Attention at a high level" (mantramindai), "The two
+ * ideas", item 3 (recompute score tiles in the backward pass instead of storing
+ * P) and "How FlashAttention Speeds Up the Attention Layer" (hassanahmed.net),
+ * the training paragraph after the online softmax; the gradients are those of
+ * standard attention (mantramindai, "Follow-up questions to expect", first
+ * question). With P = exp(scale * Q K^T - LSE) (masked entries 0):
+ *   dV = P^T dO,  dP = dO V^T,  D_i = sum_c dO_ic O_ic,  dS = P o (dP - D),
+ *   dQ = scale * dS K,  dK = scale * dS^T Q.
+ *
+ *   q, o, dout  bf16 [B, H, Nq, d]    (read; o is the forward output)
+ *   k, v        bf16 [B, H, Nkv, d]   (read)
+ *   lse         fp32 [B, H, Nq]       (read; the forward pass's LSE)
+ *   dq          bf16 [B, H, Nq, d]    (written)
+ *   dk, dv      bf16 [B, H, Nkv, d]   (written)
+ *   workspace   device, >= attn_bwd_workspace_bytes(B, H, Nq, d) bytes,
+ *               256-byte aligned; overwritten.
+ *   d in {64, 128}; causal 0 or 1 (bottom-right, as attn_fwd); B * H <= 65535.
+ *   A query row whose LSE is -inf (it sees no key) contributes nothing.
+ *   Three kernels run on `stream` in order: D and zeroing of the accumulator,
+ *   the main kernel (one CTA per 128-key block and head), and the dQ
+ *   conversion. dQ is summed with fp32 atomic adds, so its last bits may vary
+ *   from run to run; dK and dV do not.
+ */
+attn_status_t attn_bwd(const void *q, const void *k, const void *v, const void *o,
+                       const void *dout, const float *lse, void *dq, void *dk, void *dv, int B,
+                       int H, int Nq, int Nkv, int d, int causal, float scale, void *workspace,
+                       size_t workspace_bytes, void *stream);
+
+/*
  * Synchronises `stream`, then returns and clears the device status word:
  * ATTN_ERR_TIMEOUT if a kernel's pipeline wait gave up since the last call
  * (its outputs are then invalid), ATTN_ERR_CUDA if the stream reported an

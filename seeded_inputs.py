@@ -74,6 +74,15 @@ def make_qkv(B: int, H: int, Nq: int, Nkv: int, d: int, seed: int,
     return (q.to(torch.bfloat16), k.to(torch.bfloat16), v.to(torch.bfloat16))
 
 
+def make_dout(B: int, H: int, Nq: int, d: int, seed: int, device: str = "cpu"):
+    """Draw a bf16 output gradient dO [B,H,Nq,d], i.i.d. N(0,1), from its own
+    stream (``seed`` offset so that it is not a copy of Q)."""
+    g = torch.Generator(device=device)
+    g.manual_seed(seed + 7919)
+    return torch.randn((B, H, Nq, d), generator=g, device=device,
+                       dtype=torch.float32).to(torch.bfloat16)
+
+
 def make_workload(w: Workload, device: str = "cpu"):
     return make_qkv(w.B, w.H, w.Nq, w.Nkv, w.d, w.seed, device=device)
 

@@ -3,6 +3,26 @@
 The bar: O (bf16) within max-abs 1e-2 and mean-abs 1e-3 of the fp64 oracle;
 LSE (fp32) within 1e-3 absolute. Rows with no visible key must be exactly
 O = 0 and LSE = -inf on both sides.
+
+Gradients (bf16 dQ, dK, dV) are held, element by element, to an error model
+built from the oracle's fp64 quantities (see ``grad_error_bound``):
+    |g - g_ref| <= 2^-8 |g_ref| + KAPPA 2^-9 M + 1.5 |A|
+and on average to mean|g - g_ref| <= GRAD_MEAN_REL * R (R = RMS of g_ref).
+M is the quadrature magnitude of the terms each gradient sums (for dV_kc,
+sqrt(sum_i (P_ik dO_ic)^2)): the kernel rounds P and dS to bf16 (relative
+<= 2^-9, uniform, so sigma = 2^-9 M / sqrt 3) before the tensor-core products,
+and independent rounding errors add in quadrature like the terms. 2^-8 |g_ref|
+covers the bf16 rounding of the output (2^-9) twice over. A is the exact
+first-order effect of the forward output's own rounding on D = rowsum(dO o O)
+(the backward pass reads O as an input): dD_i = sum_c dO_ic (O_ic - O_ref_ic)
+shifts dS by -P dD, i.e. dQ by -scale dD (P K) and dK by -scale P^T (dD o Q).
+F (added to the dQ and dK bounds) covers the fp32 evaluation of dP - D: both
+are d-term fp32 dot products, off by at most d 2^-24 <= 2^-17 of the sum of
+absolute terms. It matters where dS cancels exactly, e.g. a row that sees one
+key (P = 1, dS = dP - D = 0, so the oracle's dQ row is 0).
+KAPPA = 8 is about 14 sigma; an emulation of exactly these roundings in fp64
+needs at most 3.7 on the shapes the tests use (gpt2-style 1K causal included).
+The mean bar: the emulated mean error is <= 1.8e-3 R on those shapes.
 """
 from __future__ import annotations
 
@@ -34,3 +54,51 @@ def compare(o_gpu, lse_gpu, o_ref, lse_ref, what=""):
     assert mean <= O_MEAN_ABS, f"{what}: mean|dO| {mean:.3e} > {O_MEAN_ABS}"
     assert ml <= LSE_MAX_ABS, f"{what}: max|dLSE| {ml:.3e} > {LSE_MAX_ABS}"
     return mx, mean, ml
+
+
+GRAD_KAPPA = 8.0
+GRAD_MEAN_REL = 4e-3
+
+
+def grad_error_bound(q, k, v, do, o_gpu, p, o_ref, causal, scale):
+    """Per-element error bounds for (dQ, dK, dV) of one head.
+
+    q, k, v, do, o_gpu: fp64 arrays of the values the kernel saw; p, o_ref: the
+    oracle's fp64 probabilities and output for this head."""
+    dp = do @ v.T
+    dsv = p * (dp - (do * o_ref).sum(1)[:, None])
+    m_dv = np.sqrt((p ** 2).T @ (do ** 2))
+    m_dk = scale * np.sqrt((dsv ** 2).T @ (q ** 2))
+    m_dq = scale * np.sqrt((dsv ** 2) @ (k ** 2))
+    dd = (do * (o_gpu - o_ref)).sum(1)
+    a_dq = scale * np.abs(dd)[:, None] * np.abs(p @ k)
+    a_dk = scale * np.abs(p.T @ (dd[:, None] * q))
+    # fp32 evaluation of dP - D (d-term dot products, worst case d 2^-24 <= 2^-17 relative)
+    f_ds = 2.0 ** -17 * p * (np.abs(do) @ np.abs(v).T + np.abs(do * o_gpu).sum(1)[:, None])
+    f_dq = scale * f_ds @ np.abs(k)
+    f_dk = scale * f_ds.T @ np.abs(q)
+    e = 2.0 ** -9
+    return (GRAD_KAPPA * e * m_dq + 1.5 * a_dq + f_dq, GRAD_KAPPA * e * m_dk + 1.5 * a_dk + f_dk,
+            GRAD_KAPPA * e * m_dv)
+
+
+def compare_grad(g_gpu, g_ref, bound, what=""):
+    """Assert |g_gpu - g_ref| <= 2^-8 |g_ref| + bound element-wise and the mean
+    bar. Returns (max over elements of err / allowed, mean|err| / R)."""
+    g_gpu = np.asarray(g_gpu, dtype=np.float64)
+    g_ref = np.asarray(g_ref, dtype=np.float64)
+    assert g_gpu.shape == g_ref.shape == bound.shape, (what, g_gpu.shape, g_ref.shape)
+    assert np.all(np.isfinite(g_gpu)), f"{what}: non-finite gradient"
+    err = np.abs(g_gpu - g_ref)
+    allowed = 2.0 ** -8 * np.abs(g_ref) + bound
+    bad = err > allowed
+    if bad.any():
+        i = np.unravel_index(int(np.argmax(err - allowed)), err.shape)
+        raise AssertionError(f"{what}: {int(bad.sum())} elements outside the error model, worst "
+                             f"at {i}: got {g_gpu[i]:.6g}, oracle {g_ref[i]:.6g}, "
+                             f"allowed |err| {allowed[i]:.3g}")
+    rms = float(np.sqrt(np.mean(g_ref ** 2)))
+    mean = float(err.mean()) / rms if rms > 0 else 0.0
+    assert mean <= GRAD_MEAN_REL, f"{what}: mean|err| {mean:.3e} R > {GRAD_MEAN_REL} R (R={rms:.3e})"
+    ratio = np.where(allowed > 0, err / np.where(allowed > 0, allowed, 1.0), 0.0)
+    return float(ratio.max()), mean

@@ -31,7 +31,7 @@ def test_header_declares_the_boundary():
     names = declared_functions()
     for want in ("attn_fwd", "attn_decode_partials", "attn_lse_merge", "attn_decode_splitkv",
                  "attn_decode_workspace_bytes", "attn_status", "attn_strerror",
-                 "attn_abi_version"):
+                 "attn_abi_version", "attn_bwd", "attn_bwd_workspace_bytes"):
         assert want in names
 
 
@@ -89,6 +89,33 @@ def test_decode_and_merge_reject_bad_arguments(ea):
     assert L.attn_decode_splitkv(p, p, p, p, p, 2, 3, 64, 128, 0.1, 8, p, need - 1, None) == 1
     assert L.attn_decode_splitkv(p, p, p, p, p, 2, 3, 64, 128, 0.1, 8, p + 16, need, None) == 3
     assert L.attn_decode_splitkv(p, p, p, p, p, 2, 3, 64, 96, 0.1, 8, p, need, None) == 2
+
+
+def test_bwd_rejects_bad_arguments_without_launching(ea):
+    L = ea.lib
+    p = 0x10000
+    ws_need = ea.attn_bwd_workspace_bytes(1, 2, 300, 128)
+    assert ws_need == (2 * 300 * 4 + 255) // 256 * 256 + 2 * 300 * 128 * 4
+    assert ea.attn_bwd_workspace_bytes(1, 2, 300, 96) == 0
+    assert ea.attn_bwd_workspace_bytes(1, 2, 0, 128) == 0
+
+    def call(ws_bytes=ws_need, **kw):
+        a = dict(dict(q=p, k=p, v=p, o=p, do=p, lse=p, dq=p, dk=p, dv=p, ws=p, B=1, H=2, Nq=300,
+                      Nkv=300, d=128, causal=1, scale=0.088), **kw)
+        return L.attn_bwd(a["q"], a["k"], a["v"], a["o"], a["do"], a["lse"], a["dq"], a["dk"],
+                          a["dv"], a["B"], a["H"], a["Nq"], a["Nkv"], a["d"], a["causal"],
+                          a["scale"], a["ws"], ws_bytes, None)
+
+    assert call(do=None) == ea.ATTN_ERR_INVALID_ARG
+    assert call(ws=None) == ea.ATTN_ERR_INVALID_ARG
+    assert call(ws_bytes=ws_need - 1) == ea.ATTN_ERR_INVALID_ARG
+    assert call(causal=2) == ea.ATTN_ERR_INVALID_ARG
+    assert call(scale=float("nan")) == ea.ATTN_ERR_INVALID_ARG
+    assert call(Nkv=0) == ea.ATTN_ERR_INVALID_ARG
+    assert call(B=70000) == ea.ATTN_ERR_INVALID_ARG
+    assert call(d=80) == ea.ATTN_ERR_UNSUPPORTED
+    assert call(dk=p + 8) == ea.ATTN_ERR_ALIGNMENT
+    assert call(ws=p + 16) == ea.ATTN_ERR_ALIGNMENT
 
 
 def test_package_fails_loudly_without_the_library(tmp_path):

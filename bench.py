@@ -10,6 +10,9 @@ Inputs are seeded i.i.d. N(0,1) bf16 (seeded_inputs.py), resident in HBM
 before timing; they exceed the 126 MB L2 (192 MB prefill + 8.6 GB decode), so
 no extra flush is needed between steps.
 
+``--workload prefill_8k_bwd`` (or another ``*_bwd``) times the backward pass
+(dQ, dK, dV) of that prefill workload instead, one attn_bwd call per step.
+
 ``--impl reference`` times the fp64 CPU oracle on a bounded sample of the same
 workloads instead (the reference arm); it never touches the GPU path.
 
@@ -81,6 +84,17 @@ def decode_partial_bytes(w):
     return decode_kv_bytes(w) + w.B * w.H * (w.d * 2 + w.num_splits * (w.d + 1) * 4)
 
 
+def bwd_flops(w):
+    """Five products per visible pair (S, dP, dV, dK, dQ), 2 d FLOP each."""
+    return 10.0 * w.d * w.B * w.H * prefill_pairs(w)
+
+
+def bwd_bytes(w):
+    """Compulsory traffic: Q, K, V, O, dO, LSE read; dQ, dK, dV written."""
+    return w.B * w.H * (3 * w.Nq * w.d * 2 + 2 * w.Nkv * w.d * 2 + 4 * w.Nq
+                        + w.Nq * w.d * 2 + 2 * w.Nkv * w.d * 2)
+
+
 def merge_bytes(w):
     return w.B * w.H * (w.num_splits * (w.d + 1) * 4 + w.d * 2 + 4)
 
@@ -148,18 +162,29 @@ class ClockSampler:
                 "reasons": sorted(reasons), "samples": len(sm)}
 
 
-def kernel_source_hash():
+# The device code each kernel's DRAM traffic depends on (its own header and the
+# PTX helpers it includes). A recorded figure is used only while these files
+# hash to the value stored beside it.
+KERNEL_SOURCES = {
+    "attn_fwd_sm100": ("fwd_sm100.cuh", "ptx_sm100.cuh", "tmem_wide.cuh"),
+    "attn_decode_partials": ("decode_sm100.cuh", "ptx_sm100.cuh"),
+    "attn_lse_merge": ("decode_sm100.cuh",),
+    "attn_bwd_sm100": ("bwd_sm100.cuh", "ptx_sm100.cuh", "tmem_wide.cuh"),
+}
+
+
+def kernel_source_hash(kernel):
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "exact_io_aware_70_b200", "csrc")
-    for f in sorted(os.listdir(csrc)):
-        if f.endswith((".cu", ".cuh")):
-            with open(os.path.join(csrc, f), "rb") as fh:
-                h.update(fh.read())
+    for f in KERNEL_SOURCES[kernel]:
+        with open(os.path.join(csrc, f), "rb") as fh:
+            h.update(fh.read())
     return h.hexdigest()[:16]
 
 
 def recorded_traffic():
-    """Per-launch DRAM traffic from the committed ncu summary, if taken on this source."""
+    """Per-launch DRAM traffic from the committed ncu summary, for each kernel
+    whose sources still hash to the value recorded with its figure."""
     path = os.path.join(ROOT, "profiles", "dram_traffic.md")
     try:
         with open(path) as fh:
@@ -167,12 +192,12 @@ def recorded_traffic():
     except OSError:
         return {}
     import re
-    m = re.search(r"source_hash:\s*([0-9a-f]+)", text)
-    if not m or m.group(1) != kernel_source_hash():
-        return {}
     out = {}
-    for row in re.findall(r"^\|\s*(attn_\w+)\s*\|\s*\w+\s*\|\s*(\d+)\s*\|", text, re.M):
-        out[row[0]] = int(row[1])
+    for name, _wl, nbytes, shash in re.findall(
+            r"^\|\s*(attn_\w+)\s*\|\s*([\w ]+?)\s*\|\s*(\d+)\s*\|\s*([0-9a-f]{16})\s*\|",
+            text, re.M):
+        if name in KERNEL_SOURCES and shash == kernel_source_hash(name):
+            out[name] = int(nbytes)
     return out
 
 
@@ -353,6 +378,163 @@ def run_reference(args):
         "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
     }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def oracle_bwd_sample(w, budget_s):
+    """Time the oracle's backward pass on leading square blocks of one head.
+
+    For a causal square head, the first n query rows see only the first n keys,
+    so the n x n leading block is itself a complete causal problem; n doubles
+    until one call takes a quarter of the budget."""
+    import oracle
+    from seeded_inputs import make_dout
+    orc = oracle.get()
+    q, k, v = make_qkv(1, 1, w.Nq, w.Nkv, w.d, w.seed)
+    do = make_dout(1, 1, w.Nq, w.d, w.seed)
+    f64 = lambda t, n: t[0, 0, :n].double().numpy()
+    n, dt, flops = 256, 0.0, 0.0
+    while True:
+        t0 = time.perf_counter()
+        orc.attn_bwd_head_f64(f64(q, n), f64(k, n), f64(v, n), f64(do, n), w.causal, w.scale)
+        dt = time.perf_counter() - t0
+        flops = 10.0 * w.d * (n * (n + 1) // 2 if w.causal else n * n)
+        if dt > budget_s / 4 or 2 * n > min(w.Nq, w.Nkv):
+            break
+        n *= 2
+    return {"flops": flops, "seconds": dt, "n": n, "cores": orc.num_threads()}
+
+
+def run_bwd(args):
+    """Backward pass (dQ, dK, dV) of a prefill workload: O and LSE come from one
+    untimed forward call; each step is one attn_bwd call (three kernels)."""
+    import torch
+    import torch.distributed as dist
+
+    import exact_io_aware_70_b200 as ea
+    from exact_io_aware_70_b200.replicas import max_over_ranks, replica_workload
+    from seeded_inputs import make_dout
+
+    ws, rank, local = dist_env()
+    torch.cuda.set_device(local)
+    if ws > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    dev = torch.device("cuda", local)
+    stream = torch.cuda.current_stream()
+    sp = stream.cuda_stream
+    L = ea.lib
+    w = _maybe_batch(WORKLOADS[args.workload[:-len("_bwd")]], args.batch)
+    wr = replica_workload(w, rank)
+    q, k, v = make_workload(wr, device="cuda")
+    do = make_dout(w.B, w.H, w.Nq, w.d, wr.seed, device="cuda")
+    o = torch.empty_like(q)
+    lse = torch.empty((w.B, w.H, w.Nq), dtype=torch.float32, device=dev)
+    ea.attn_fwd(q, k, v, o, lse, w.causal, w.scale)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    work = torch.empty(ea.attn_bwd_workspace_bytes(w.B, w.H, w.Nq, w.d), dtype=torch.uint8,
+                       device=dev)
+    args_c = (q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), do.data_ptr(),
+              lse.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), w.B, w.H, w.Nq, w.Nkv,
+              w.d, int(w.causal), w.scale, work.data_ptr(), work.numel(), sp)
+
+    def step():
+        rc = L.attn_bwd(*args_c)
+        if rc != 0:
+            raise RuntimeError(f"attn_bwd: {ea.attn_strerror(rc)}")
+
+    for _ in range(args.warmup):
+        step()
+    if ea.attn_status() != 0:
+        raise RuntimeError("device status reported an error during warm-up")
+    K = args.steps
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(K + 1)]
+    with ClockSampler(local) as clk:
+        if ws > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+        for s in range(K):
+            ev[s].record(stream)
+            step()
+        ev[K].record(stream)
+        torch.cuda.synchronize()
+        if ws > 1:
+            dist.barrier()
+    if ea.attn_status() != 0:
+        raise RuntimeError("device status reported an error in the timed region")
+    total_ms = ev[0].elapsed_time(ev[K])
+    call_ms = statistics.mean(ev[s].elapsed_time(ev[s + 1]) for s in range(K))
+
+    e2e = None
+    if not args.no_e2e:
+        hin = [t.cpu().pin_memory() for t in (q, k, v, o, do, lse)]
+        hout = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in (dq, dk, dv)]
+        h2d = sum(t.numel() * t.element_size() for t in hin)
+        d2h = sum(t.numel() * t.element_size() for t in hout)
+
+        def e2e_step():
+            for dst, src in zip((q, k, v, o, do, lse), hin):
+                dst.copy_(src, non_blocking=True)
+            ea.attn_bwd(q, k, v, o, do, lse, dq, dk, dv, w.causal, w.scale, work)
+            for dst, src in zip(hout, (dq, dk, dv)):
+                dst.copy_(src, non_blocking=True)
+
+        e2e_step()
+        torch.cuda.synchronize()
+        E = max(2, min(K, 3))
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(E):
+            e2e_step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        ems = e0.elapsed_time(e1) / E
+        if ea.attn_status() != 0:
+            raise RuntimeError("device status reported an error in the e2e region")
+        e2e = {"value": None, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
+               "d2h_bytes_per_step": d2h, "ms_per_step": ems, "steps": E,
+               "path": "pinned host -> copy -> attn_bwd -> copy back, per step, CUDA events"}
+    vals = max_over_ranks([total_ms, call_ms] + ([e2e["ms_per_step"]] if e2e else []), device=dev)
+    total_ms, call_ms = vals[0], vals[1]
+    if e2e:
+        e2e["ms_per_step"] = vals[2]
+        e2e["value"] = ws * bwd_flops(w) / (vals[2] * 1e-3) / 1e12
+    if ws > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return 0
+    pk = peaks()
+    a = bwd_flops(w) / (call_ms * 1e-3) / 1e12
+    roof = {"kernel": "attn_bwd (preprocess + attn_bwd_sm100 + postprocess, timed as one call)",
+            "bound": "tensor", "achieved": a, "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
+            "frac": a / pk["bf16_tflops"], "frac_of_sustained": a / pk["bf16_tflops_sustained"],
+            "traffic": recorded_traffic().get("attn_bwd_sm100"),
+            "algorithmic_bytes": bwd_bytes(w), "algorithmic_flops": bwd_flops(w), "ms": call_ms}
+    line = {
+        "metric": "attn bwd TFLOP/s & % BF16 tensor peak",
+        "value": ws * a, "unit": "TFLOP/s", "n_gpus": ws, "steps": K, "warmup": args.warmup,
+        "ms_per_step": total_ms / K, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": args.workload, "B": w.B, "H": w.H, "N": w.Nq, "d": w.d,
+                   "causal": w.causal, "flop_per_step": bwd_flops(w),
+                   "l2": "inputs larger than L2 (126 MB); no flush" if not args.batch else
+                         "reduced batch for profiling",
+                   "parallelism": f"replicas x{ws}" if ws > 1 else "1 GPU"},
+        "roofline": roof,
+        "peaks": dict(pk, note="of measured" if pk["source"] == "measured" else "of fallback"),
+        "clocks": clk.summary(max_mhz_default=1965.0),
+        "gpu_launches": 3 * K, "e2e": e2e,
+    }
+    if ws == 1 and not args.no_cpu_baseline:
+        cb = oracle_bwd_sample(w, args.cpu_budget)
+        line["cpu_baseline"] = {
+            "value": cb["flops"] / cb["seconds"] / 1e12, "unit": "TFLOP/s", "cores": cb["cores"],
+            "kind": "oracle",
+            "sample": f"fp64 oracle backward of the leading {cb['n']}x{cb['n']} block of one "
+                      f"head ({cb['flops'] / 1e9:.1f} GFLOP in {cb['seconds']:.2f} s)"}
     print(json.dumps(line), flush=True)
     return 0
 
@@ -638,8 +820,10 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="step",
                     choices=["step", "prefill_8k", "prefill_16k", "gpt2_1k", "tiny", "decode_32k",
-                             "decode_32k_paged"],
-                    help="step = prefill_8k + decode_32k (the default bench line)")
+                             "decode_32k_paged", "prefill_8k_bwd", "prefill_16k_bwd",
+                             "gpt2_1k_bwd"],
+                    help="step = prefill_8k + decode_32k (the default bench line); "
+                         "*_bwd = the backward pass of that prefill workload")
     ap.add_argument("--batch", type=int, default=0,
                     help="override the batch size (small profiling captures only)")
     ap.add_argument("--no-e2e", action="store_true")
@@ -653,6 +837,8 @@ def main():
         args.warmup = 3
     if args.impl == "reference":
         return run_reference(args)
+    if args.workload.endswith("_bwd"):
+        return run_bwd(args)
     return run_ours(args)
 
 

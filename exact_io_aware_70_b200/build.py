@@ -57,6 +57,10 @@ def build(force: bool = False, verbose: bool = False) -> str:
 # Fewer at launch would make the softmax warpgroups' increase wait forever, so
 # the build refuses to produce such a library.
 FWD_LAUNCH_REGS = 168
+# The backward kernel runs 10 warps per CTA; registers are split between the
+# SM's four schedulers, so three warps on one scheduler cap a thread at 168
+# registers. More would make every launch fail ("too many resources").
+BWD_MAX_REGS = 168
 
 
 def check_register_budget(ptxas_log: str) -> None:
@@ -68,6 +72,10 @@ def check_register_budget(ptxas_log: str) -> None:
             current = m.group(1)
             continue
         m = re.search(r"Used (\d+) registers", line)
+        if m and current and "attn_bwd_sm100_kernel" in current and int(m.group(1)) > BWD_MAX_REGS:
+            os.remove(LIB)
+            raise RuntimeError(f"{current} uses {m.group(1)} registers, more than "
+                               f"{BWD_MAX_REGS}: its 320-thread launch would fail")
         if m and current and "attn_fwd_sm100_kernel" in current:
             seen += 1
             if int(m.group(1)) != FWD_LAUNCH_REGS:

@@ -19,6 +19,7 @@ _c_long = ctypes.c_long
 _dp = ctypes.POINTER(ctypes.c_double)
 _fp = ctypes.POINTER(ctypes.c_float)
 _u16p = ctypes.POINTER(ctypes.c_uint16)
+_u8p = ctypes.POINTER(ctypes.c_uint8)
 _i64p = ctypes.POINTER(ctypes.c_int64)
 
 
@@ -55,6 +56,10 @@ class Oracle:
         lib.oracle_attn_bwd_bf16.argtypes = [_u16p, _u16p, _u16p, _u16p, _c_long, _c_long,
                                              _c_long, _c_long, _c_long, ctypes.c_int,
                                              ctypes.c_double, _dp, _dp, _dp]
+        lib.oracle_e4m3_decode.argtypes = [_u8p, _c_long, _dp]
+        lib.oracle_attn_fwd_fp8.argtypes = [_u8p, _u8p, _u8p, _fp, _fp, _fp, _c_long, _c_long,
+                                            _c_long, _c_long, _c_long, ctypes.c_int,
+                                            ctypes.c_double, _dp, _dp]
         lib.oracle_num_threads.restype = ctypes.c_int
         lib.oracle_set_num_threads.argtypes = [ctypes.c_int]
         self.lib = lib
@@ -148,6 +153,30 @@ class Oracle:
         if rc:
             raise RuntimeError("oracle_attn_bwd_bf16 failed")
         return dq, dk, dv
+
+    def e4m3_decode(self, codes):
+        """Values of e4m3 codes (uint8 array) as doubles, from the format's definition."""
+        c = np.ascontiguousarray(codes, dtype=np.uint8)
+        out = np.zeros(c.shape)
+        self.lib.oracle_e4m3_decode(_ptr(c, _u8p), c.size, _ptr(out, _dp))
+        return out
+
+    def attn_fwd_fp8(self, q_codes, k_codes, v_codes, q_descale, k_descale, v_descale,
+                     causal: bool, scale: float):
+        """e4m3 codes [B,H,N,d] (uint8) and fp32 descales [B,H] -> (O f64, LSE f64)."""
+        B, H, Nq, d = q_codes.shape
+        Nkv = k_codes.shape[2]
+        q, k, v = (np.ascontiguousarray(x, dtype=np.uint8) for x in (q_codes, k_codes, v_codes))
+        qd, kd, vd = (np.ascontiguousarray(x, dtype=np.float32).reshape(B * H)
+                      for x in (q_descale, k_descale, v_descale))
+        o, lse = np.zeros((B, H, Nq, d)), np.zeros((B, H, Nq))
+        rc = self.lib.oracle_attn_fwd_fp8(_ptr(q, _u8p), _ptr(k, _u8p), _ptr(v, _u8p),
+                                          _ptr(qd, _fp), _ptr(kd, _fp), _ptr(vd, _fp), B, H, Nq,
+                                          Nkv, d, int(causal), float(scale), _ptr(o, _dp),
+                                          _ptr(lse, _dp))
+        if rc:
+            raise RuntimeError("oracle_attn_fwd_fp8 failed")
+        return o, lse
 
     def decode_paged_bf16(self, q_bits, k_cache_bits, v_cache_bits, block_table, seq_lens,
                           scale: float):

@@ -490,6 +490,71 @@ int oracle_attn_bwd_bf16(const uint16_t *q, const uint16_t *k, const uint16_t *v
     return 0;
 }
 
+/*
+ * 8-bit inputs. The pages name an FP8 path (mantramindai "Versions";
+ * hassanahmed.net, the FlashAttention-3 paragraph) but no format; the reading
+ * used here: OCP FP8 E4M3 codes with one descale factor per (b, h) and
+ * tensor, a code c standing for descale * value(c). The oracle decodes each
+ * code from the format's definition and evaluates the same exact attention
+ * on the decoded values; how a kernel rounds P internally is not its concern.
+ *
+ * E4M3: bit 7 sign, bits 3-6 exponent with bias 7, bits 0-2 mantissa. An
+ * exponent field of 0 is subnormal (mantissa/8 * 2^-6); exponent 15 with
+ * mantissa 7 is NaN; there are no infinities (so 0x7E = 448 is the largest).
+ */
+static double e4m3_to_double(uint8_t c) {
+    const int sign = c >> 7, e = (c >> 3) & 15, m = c & 7;
+    if (e == 15 && m == 7) return NAN;
+#if ORACLE_MUTANT == 14 /* exponent bias 8 instead of 7 */
+    const int bias = 8;
+#else
+    const int bias = 7;
+#endif
+    const double mag = (e == 0) ? ldexp((double)m / 8.0, 1 - bias)
+                                : ldexp(1.0 + (double)m / 8.0, e - bias);
+    return sign ? -mag : mag;
+}
+
+/* decoded values of n codes (for the pins) */
+void oracle_e4m3_decode(const uint8_t *codes, long n, double *out) {
+    for (long i = 0; i < n; ++i) out[i] = e4m3_to_double(codes[i]);
+}
+
+static double *widen_e4m3(const uint8_t *src, size_t n, double descale) {
+    double *dst = (double *)malloc(n * sizeof(double));
+    if (!dst) return NULL;
+    for (size_t i = 0; i < n; ++i) dst[i] = descale * e4m3_to_double(src[i]);
+    return dst;
+}
+
+/*
+ * Exact attention on e4m3 inputs [B, H, N, d] with descale factors [B, H]
+ * (fp32, widened exactly). o [B, H, Nq, d] and lse [B, H, Nq] are double.
+ */
+int oracle_attn_fwd_fp8(const uint8_t *q, const uint8_t *k, const uint8_t *v,
+                        const float *q_descale, const float *k_descale,
+                        const float *v_descale, long B, long H, long Nq, long Nkv, long d,
+                        int causal, double scale, double *o, double *lse) {
+    if (B < 0 || H < 0 || Nq < 0 || Nkv < 0 || d <= 0) return -1;
+    for (long bh = 0; bh < B * H; ++bh) {
+#if ORACLE_MUTANT == 15 /* V's descale factor ignored */
+        const double dv = 1.0;
+#else
+        const double dv = (double)v_descale[bh];
+#endif
+        double *qh = widen_e4m3(q + bh * Nq * d, (size_t)(Nq * d), (double)q_descale[bh]);
+        double *kh = widen_e4m3(k + bh * Nkv * d, (size_t)(Nkv * d), (double)k_descale[bh]);
+        double *vh = widen_e4m3(v + bh * Nkv * d, (size_t)(Nkv * d), dv);
+        int rc = (qh && kh && vh) ? 0 : -1;
+        if (rc == 0)
+            rc = oracle_attn_head_f64(qh, kh, vh, Nq, Nkv, d, causal, scale,
+                                      o + bh * Nq * d, lse + bh * Nq, NULL);
+        free(qh); free(kh); free(vh);
+        if (rc) return rc;
+    }
+    return 0;
+}
+
 /* number of OpenMP threads the oracle will use (1 without OpenMP) */
 int oracle_num_threads(void) {
 #ifdef _OPENMP

@@ -83,6 +83,29 @@ def make_dout(B: int, H: int, Nq: int, d: int, seed: int, device: str = "cpu"):
                        dtype=torch.float32).to(torch.bfloat16)
 
 
+def make_qkv_fp8(B: int, H: int, Nq: int, Nkv: int, d: int, seed: int, device: str = "cpu"):
+    """e4m3 versions of make_qkv's draws: per (b, h) and tensor, descale =
+    max|x| / 448 (rounded to fp32) and code = e4m3(x / descale) (torch's
+    round-to-nearest cast, clamped to the format's +-448). Returns the codes
+    [B,H,N,d] as torch.float8_e4m3fn and the descales [B,H] fp32."""
+    g = torch.Generator(device=device)
+    g.manual_seed(seed)
+    out = []
+    for n in (Nq, Nkv, Nkv):
+        x = torch.randn((B, H, n, d), generator=g, device=device, dtype=torch.float32)
+        ds = (x.abs().amax(dim=(2, 3)) / 448.0).clamp_min(1e-30)
+        codes = (x / ds[:, :, None, None]).clamp(-448.0, 448.0).to(torch.float8_e4m3fn)
+        out += [codes, ds.contiguous()]
+    q8, qd, k8, kd, v8, vd = out
+    return q8, k8, v8, qd, kd, vd
+
+
+def fp8_codes(t: torch.Tensor):
+    """The raw uint8 codes of a contiguous float8_e4m3fn CPU tensor, as numpy."""
+    assert t.dtype == torch.float8_e4m3fn
+    return t.contiguous().view(torch.uint8).numpy()
+
+
 def make_workload(w: Workload, device: str = "cpu"):
     return make_qkv(w.B, w.H, w.Nq, w.Nkv, w.d, w.seed, device=device)
 

@@ -416,6 +416,48 @@ def pin_bwd_invariants(orc):
     _close(dv, np.tile(do.sum(axis=0) / Nkv, (Nkv, 1)), 1e-12, "uniform weights dV")
 
 
+# ---------------------------------------------------------------------------
+# 9. e4m3 (8-bit) inputs
+# ---------------------------------------------------------------------------
+def pin_e4m3_decode(orc):
+    """All 256 codes against torch's float8_e4m3fn widening (a library routine),
+    plus values fixed by the format's definition."""
+    codes = np.arange(256, dtype=np.uint8)
+    got = orc.e4m3_decode(codes)
+    ref = torch.from_numpy(codes.copy()).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    nan = np.isnan(ref)
+    assert np.array_equal(np.isnan(got), nan), "e4m3 NaN codes"
+    _close(got[~nan], ref[~nan], 0.0, "e4m3 decode vs torch")
+    hand = {0x00: 0.0, 0x01: 2.0 ** -9, 0x07: 7 * 2.0 ** -9, 0x08: 2.0 ** -6, 0x38: 1.0,
+            0x39: 1.125, 0x40: 2.0, 0x7E: 448.0, 0xB8: -1.0, 0xFE: -448.0}
+    for c, val in hand.items():
+        _close(got[c], val, 0.0, f"e4m3 code {c:#04x}")
+    assert np.isnan(got[0x7F]) and np.isnan(got[0xFF])
+
+
+def pin_fp8_entry(orc):
+    """The 8-bit entry equals the double entry on the values the codes and
+    descale factors stand for (decoded here by torch, not by the oracle)."""
+    rng = np.random.default_rng(7)
+    B, H, Nq, Nkv, d = 1, 2, 9, 13, 16
+    for causal in (False, True):
+        q8, k8, v8 = (rng.integers(0, 256, size=(B, H, n, d), dtype=np.uint8)
+                      for n in (Nq, Nkv, Nkv))
+        for t in (q8, k8, v8):        # keep the codes finite (no NaN pattern)
+            t[(t & 0x7F) == 0x7F] = 0x38
+        qd, kd, vd = (rng.uniform(0.01, 0.1, size=(B, H)).astype(np.float32) for _ in range(3))
+        o, lse = orc.attn_fwd_fp8(q8, k8, v8, qd, kd, vd, causal, 0.25)
+
+        def val(c, ds, h):
+            return (torch.from_numpy(c[0, h].copy()).view(torch.float8_e4m3fn)
+                    .to(torch.float64).numpy() * float(ds[0, h]))
+        for h in range(H):
+            ro, rl = orc.attn_head_f64(val(q8, qd, h), val(k8, kd, h), val(v8, vd, h), causal,
+                                       0.25)
+            _close(o[0, h], ro, 1e-12, f"fp8 entry O head {h}")
+            _close(lse[0, h], rl, 1e-12, f"fp8 entry LSE head {h}")
+
+
 ALL_PINS = [
     pin_worked_example, pin_golden_cases, pin_probabilities, pin_constant_values,
     pin_identical_keys, pin_zero_query, pin_causal_first_row, pin_key_permutation,
@@ -423,4 +465,5 @@ ALL_PINS = [
     pin_partials_are_chunk_attention, pin_merge_batched_matches_single, pin_bf16_entry,
     pin_paged_matches_contiguous, pin_paged_golden,
     pin_bwd_torch_autograd, pin_bwd_finite_differences, pin_bwd_invariants,
+    pin_e4m3_decode, pin_fp8_entry,
 ]

@@ -4,7 +4,9 @@ The oracle source has ORACLE_MUTANT switches, each planting one plausible bug
 (dropped scale, wrong key index, off-by-one or mis-aligned causal mask, sign
 error in the exponent, dropped normalisation, LSE without the max term,
 transposed V, unnormalised merge weights, a paged decode that ignores its block
-table or reads past the sequence). Building each variant and running
+table or reads past the sequence, a backward pass without the D term or the
+dK scale, an e4m3 decoder with the wrong exponent bias, an 8-bit entry that
+ignores V's descale factor). Building each variant and running
 the pins shows the pins would notice that mistake in the real oracle.
 """
 import pytest
@@ -26,6 +28,8 @@ MUTANTS = {
     11: "paged decode reads one token past the sequence",
     12: "backward drops the D term",
     13: "backward dK without the scale",
+    14: "e4m3 exponent bias 8",
+    15: "e4m3 V descale ignored",
 }
 
 

@@ -7,6 +7,9 @@ has not been built; there is no fallback implementation.
 
 Entry points (same names as the C ABI):
   attn_fwd(q, k, v, o, lse, causal, scale)            prefill forward, O and LSE
+  attn_fwd_fp8(q, k, v, q_descale, k_descale, v_descale, o, lse, causal, scale)
+  attn_bwd(q, k, v, o, dout, lse, dq, dk, dv, causal, scale, workspace)
+  attn_bwd_workspace_bytes(B, H, Nq, d)
   attn_decode_partials(q, k, v, o_part, lse_part, scale, num_splits)
   attn_lse_merge(o_part, lse_part, o, lse)
   attn_decode_splitkv(q, k, v, o, lse, scale, num_splits, workspace)
@@ -44,6 +47,8 @@ lib.attn_strerror.restype = ctypes.c_char_p
 lib.attn_strerror.argtypes = [_i]
 lib.attn_fwd.restype = _i
 lib.attn_fwd.argtypes = [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _f, _vp]
+lib.attn_fwd_fp8.restype = _i
+lib.attn_fwd_fp8.argtypes = [_vp] * 8 + [_i] * 6 + [_f, _vp]
 lib.attn_decode_partials.restype = _i
 lib.attn_decode_partials.argtypes = [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _f, _i, _vp]
 lib.attn_lse_merge.restype = _i
@@ -117,6 +122,27 @@ def attn_fwd(q, k, v, o, lse, causal: bool, scale: float, stream=None) -> None:
                         _tensor(v, torch.bfloat16, "v"), _tensor(o, torch.bfloat16, "o"),
                         _tensor(lse, torch.float32, "lse"), B, H, Nq, Nkv, d, int(bool(causal)),
                         float(scale), _stream(stream)), "attn_fwd")
+
+
+def attn_fwd_fp8(q, k, v, q_descale, k_descale, v_descale, o, lse, causal: bool, scale: float,
+                 stream=None) -> None:
+    """O and LSE from e4m3 inputs. q [B,H,Nq,128], k/v [B,H,Nkv,128] torch.float8_e4m3fn;
+    *_descale [B,H] fp32; o [B,H,Nq,128] bf16; lse [B,H,Nq] fp32."""
+    import torch
+    B, H, Nq, d = q.shape
+    Nkv = k.shape[2]
+    if tuple(k.shape) != (B, H, Nkv, d) or tuple(v.shape) != (B, H, Nkv, d) \
+            or tuple(o.shape) != (B, H, Nq, d) or tuple(lse.shape) != (B, H, Nq) \
+            or any(tuple(t.shape) != (B, H) for t in (q_descale, k_descale, v_descale)):
+        raise ValueError("attn_fwd_fp8: inconsistent shapes")
+    f8 = torch.float8_e4m3fn
+    _check(lib.attn_fwd_fp8(_tensor(q, f8, "q"), _tensor(k, f8, "k"), _tensor(v, f8, "v"),
+                            _tensor(q_descale, torch.float32, "q_descale"),
+                            _tensor(k_descale, torch.float32, "k_descale"),
+                            _tensor(v_descale, torch.float32, "v_descale"),
+                            _tensor(o, torch.bfloat16, "o"), _tensor(lse, torch.float32, "lse"),
+                            B, H, Nq, Nkv, d, int(bool(causal)), float(scale), _stream(stream)),
+           "attn_fwd_fp8")
 
 
 def attn_decode_partials(q, k, v, o_part, lse_part, scale: float, num_splits: int,

@@ -84,9 +84,24 @@ bool encode_bf16_map(CUtensorMap* map, const void* base, int BH, int N, int D) {
     return r == CUDA_SUCCESS;
 }
 
+// Tensor map over an 8-bit tensor viewed as [BH][N][D] with D = 128: box =
+// 128 rows x 128 bytes, 128-byte swizzle, out-of-range rows read as zero.
+bool encode_u8_map(CUtensorMap* map, const void* base, int BH, int N, int D) {
+    EncodeTiledFn enc = get_encode_fn();
+    if (!enc) return false;
+    cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)N, (cuuint64_t)BH};
+    cuuint64_t strides[2] = {(cuuint64_t)D, (cuuint64_t)N * D};
+    cuuint32_t box[3] = {128, 128, 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(base), dims, strides,
+                     box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
 struct DeviceInfo {
     int sms = 0;
-    bool fwd_attr_set[4] = {false, false, false, false};
+    bool fwd_attr_set[6] = {false, false, false, false, false, false};
     bool bwd_attr_set[4] = {false, false, false, false};
 };
 DeviceInfo g_dev[64];
@@ -98,13 +113,13 @@ int current_device() {
     return dev;
 }
 
-template <int D, bool CAUSAL>
+template <int D, bool CAUSAL, bool FP8 = false>
 attn_status_t launch_fwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                          const FwdParams& p, cudaStream_t stream) {
-    using T = FwdTraits<D>;
+    using T = FwdTraits<D, FP8>;
     const int dev = current_device();
     if (dev < 0 || dev >= 64) return ATTN_ERR_CUDA;
-    auto kern = attn_fwd_sm100_kernel<D, CAUSAL>;
+    auto kern = attn_fwd_sm100_kernel<D, CAUSAL, FP8>;
     int sms;
     {
         std::lock_guard<std::mutex> lk(g_dev_mu);
@@ -112,7 +127,7 @@ attn_status_t launch_fwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUt
         if (di.sms == 0 &&
             cudaDeviceGetAttribute(&di.sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
             return ATTN_ERR_CUDA;
-        const int slot = (D == 128 ? 2 : 0) + (CAUSAL ? 1 : 0);
+        const int slot = (FP8 ? 4 : (D == 128 ? 2 : 0)) + (CAUSAL ? 1 : 0);
         if (!di.fwd_attr_set[slot]) {
             if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                      T::kSmemBytes) != cudaSuccess)
@@ -206,6 +221,7 @@ attn_status_t attn_fwd(const void* q, const void* k, const void* v, void* o, flo
     FwdParams p;
     p.o = static_cast<uint16_t*>(o);
     p.lse = lse;
+    p.q_descale = p.k_descale = p.v_descale = nullptr;
     p.BH = BH;
     p.Nq = Nq;
     p.Nkv = Nkv;
@@ -220,6 +236,45 @@ attn_status_t attn_fwd(const void* q, const void* k, const void* v, void* o, flo
                       : launch_fwd<128, false>(tq, tk, tv, p, st);
     return causal ? launch_fwd<64, true>(tq, tk, tv, p, st)
                   : launch_fwd<64, false>(tq, tk, tv, p, st);
+}
+
+attn_status_t attn_fwd_fp8(const void* q, const void* k, const void* v, const float* q_descale,
+                           const float* k_descale, const float* v_descale, void* o, float* lse,
+                           int B, int H, int Nq, int Nkv, int d, int causal, float scale,
+                           void* stream) {
+    if (!q || !k || !v || !q_descale || !k_descale || !v_descale || !o || !lse)
+        return ATTN_ERR_INVALID_ARG;
+    if (causal != 0 && causal != 1) return ATTN_ERR_INVALID_ARG;
+    if (!(scale > 0.f) || !std::isfinite(scale)) return ATTN_ERR_INVALID_ARG;
+    attn_status_t s = check_sizes(B, H, Nq, Nkv);
+    if (s != ATTN_OK) return s;
+    if (d != 128) return ATTN_ERR_UNSUPPORTED;
+    if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) ||
+        !aligned(lse, 4) || !aligned(q_descale, 4) || !aligned(k_descale, 4) ||
+        !aligned(v_descale, 4))
+        return ATTN_ERR_ALIGNMENT;
+    const int BH = B * H;
+    CUtensorMap tq, tk, tv;
+    if (!encode_u8_map(&tq, q, BH, Nq, d) || !encode_u8_map(&tk, k, BH, Nkv, d) ||
+        !encode_u8_map(&tv, v, BH, Nkv, d))
+        return ATTN_ERR_CUDA;
+    FwdParams p;
+    p.o = static_cast<uint16_t*>(o);
+    p.lse = lse;
+    p.q_descale = q_descale;
+    p.k_descale = k_descale;
+    p.v_descale = v_descale;
+    p.BH = BH;
+    p.Nq = Nq;
+    p.Nkv = Nkv;
+    p.num_qb = (Nq + 255) / 256;
+    const long long units = (long long)BH * p.num_qb;
+    if (units > (1ll << 30)) return ATTN_ERR_INVALID_ARG;
+    p.num_units = (int)units;
+    p.scale_log2 = scale * kLog2e;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    return causal ? launch_fwd<128, true, true>(tq, tk, tv, p, st)
+                  : launch_fwd<128, false, true>(tq, tk, tv, p, st);
 }
 
 attn_status_t attn_decode_partials(const void* q, const void* k, const void* v, float* o_part,

@@ -70,6 +70,11 @@ namespace eattn {
 struct FwdParams {
     uint16_t* o;        // bf16 [BH, Nq, D]
     float* lse;         // fp32 [BH, Nq]
+    // e4m3 inputs only: per (batch*head) factors that turn the stored codes
+    // into values (x = descale * code); null for bf16 inputs
+    const float* q_descale;
+    const float* k_descale;
+    const float* v_descale;
     int BH;             // batch * heads
     int Nq, Nkv;
     int num_qb;         // ceil(Nq / 256)
@@ -95,14 +100,30 @@ struct FwdParams {
 #define EATTN_SPLIT_P 0
 #endif
 
-template <int D>
+// FP8 = true: Q, K, V are e4m3 codes with per-(batch*head) descale factors;
+// S and P V run as tcgen05.mma kind::f8f6f4 (K = 32 per instruction), P is
+// rounded to e4m3 in tensor memory. Head dim 128 only (a 128-byte row).
+template <int D, bool FP8 = false>
 struct FwdTraits {
     static_assert(D == 64 || D == 128, "head dim 64 or 128");
+    static_assert(!FP8 || D == 128, "e4m3 inputs: head dim 128");
+    static constexpr int kElemBytes = FP8 ? 1 : 2;
     static constexpr int kRows = 128;                     // rows of a Q, K or V tile
-    static constexpr int kPanelBytes = 128 * 64 * 2;      // 128 rows x 64 bf16 (one swizzle panel)
-    static constexpr int kPanels = D / 64;
+    static constexpr int kPanelBytes = 128 * 128;         // 128 rows x 128 bytes (one swizzle panel)
+    static constexpr int kPanelElems = 128 / kElemBytes;  // elements of a row in one panel
+    static constexpr int kPanels = D * kElemBytes / 128;
     static constexpr int kTileBytes = kPanels * kPanelBytes;
-    static constexpr int kSlots = (D == 128) ? EATTN_KV_SLOTS_D128 : 8;   // K/V ring depth (tiles)
+    static constexpr int kKSteps = D * kElemBytes / 32;   // 32-byte K steps of S = Q K^T
+    static constexpr int kPvSteps = FP8 ? 4 : 8;          // MMAs of P V per 128 keys
+    static constexpr int kPvRowBytes = FP8 ? 4096 : 2048; // V bytes one P V MMA consumes
+    // e4m3 P: exponents are taken against (reference max - kShift), so a row's
+    // largest values of P lie in [2^6, 2^8] and e4m3's subnormal range (below
+    // 2^-6) only holds values under 2^-12 of the row maximum; the lazy-rescale
+    // threshold is lowered so P never exceeds 2^8 (< 448, the e4m3 maximum).
+    // The shift cancels in O = acc / l and is taken out of the LSE.
+    static constexpr float kShift = FP8 ? 6.0f : 0.0f;
+    static constexpr float kLazy = FP8 ? 2.0f : 8.0f;
+    static constexpr int kSlots = FP8 ? 8 : ((D == 128) ? EATTN_KV_SLOTS_D128 : 8);   // K/V ring depth
     static_assert(kSlots >= 2, "the ring holds K_j and V_j at once");
     static_assert(!EATTN_KV_PAIR_BARRIER || kSlots % 2 == 0, "K/V pairs need an even ring");
     static constexpr int kThreads = 384;                  // 3 warpgroups
@@ -215,12 +236,12 @@ __device__ __forceinline__ bool role_wait(uint32_t bar, uint32_t parity, volatil
 
 // ----------------------------------------------------------- TMA producer --
 // Run by the whole producer warp with converged control flow; lane 0 issues.
-template <int D, bool CAUSAL>
+template <int D, bool CAUSAL, bool FP8>
 __device__ void fwd_producer(const FwdParams& p, const CUtensorMap* tq, const CUtensorMap* tk,
                              const CUtensorMap* tv, uint32_t sQ, uint32_t sKV,
-                             const FwdBars<FwdTraits<D>::kSlots>& b, uint32_t leader,
+                             const FwdBars<FwdTraits<D, FP8>::kSlots>& b, uint32_t leader,
                              volatile int* abort_flag) {
-    using T = FwdTraits<D>;
+    using T = FwdTraits<D, FP8>;
     const uint64_t pol_q = l2_policy_evict_first();
     const uint64_t pol_kv = l2_policy_evict_last();
     uint32_t kv_iter = 0;
@@ -235,11 +256,11 @@ __device__ void fwd_producer(const FwdParams& p, const CUtensorMap* tq, const CU
             for (int pn = 0; pn < T::kPanels; ++pn)
                 if (EATTN_FWD_L2_HINTS)
                     tma_load_3d_hint_w(sQ + t * T::kTileBytes + pn * T::kPanelBytes, tq,
-                                       b.q_full(t), pn * 64, x.qb * 256 + t * 128, x.bh, pol_q,
-                                       leader);
+                                       b.q_full(t), pn * T::kPanelElems, x.qb * 256 + t * 128,
+                                       x.bh, pol_q, leader);
                 else
                     tma_load_3d_w(sQ + t * T::kTileBytes + pn * T::kPanelBytes, tq, b.q_full(t),
-                                  pn * 64, x.qb * 256 + t * 128, x.bh, leader);
+                                  pn * T::kPanelElems, x.qb * 256 + t * 128, x.bh, leader);
             ++q_issued[t];
         }
         for (int j = 0; j < x.nmax; ++j) {
@@ -260,11 +281,12 @@ __device__ void fwd_producer(const FwdParams& p, const CUtensorMap* tq, const CU
                 for (int pn = 0; pn < T::kPanels; ++pn)
                     if (EATTN_FWD_L2_HINTS)
                         tma_load_3d_hint_w(sKV + slot * T::kTileBytes + pn * T::kPanelBytes,
-                                           which ? tv : tk, fbar, pn * 64, j * 128, x.bh, pol_kv,
-                                           leader);
+                                           which ? tv : tk, fbar, pn * T::kPanelElems, j * 128,
+                                           x.bh, pol_kv, leader);
                     else
                         tma_load_3d_w(sKV + slot * T::kTileBytes + pn * T::kPanelBytes,
-                                      which ? tv : tk, fbar, pn * 64, j * 128, x.bh, leader);
+                                      which ? tv : tk, fbar, pn * T::kPanelElems, j * 128, x.bh,
+                                      leader);
                 ++kv_iter;
             }
         }
@@ -288,38 +310,50 @@ fail: {
 // Descriptor bases are computed once; an operand at byte offset `off` from a
 // base is the base plus off >> 4 (the start-address field never overflows:
 // shared memory addresses are below 2^18).
-template <int D>
+template <int D, bool FP8>
 __device__ __forceinline__ void fwd_issue_s(uint32_t tmem_s, uint64_t dq, uint64_t dk,
                                             uint32_t leader) {
-    using T = FwdTraits<D>;
-    constexpr uint32_t idesc = idesc_bf16_f32(128, 128, false);
+    using T = FwdTraits<D, FP8>;
+    constexpr uint32_t idesc =
+        FP8 ? idesc_e4m3_f32(128, 128, false) : idesc_bf16_f32(128, 128, false);
 #pragma unroll
-    for (int kk = 0; kk < D / 16; ++kk) {
+    for (int kk = 0; kk < T::kKSteps; ++kk) {
+        // one MMA consumes 32 bytes of every row (16 bf16 or 32 e4m3 elements)
         const uint64_t off = ((kk / 4) * T::kPanelBytes + (kk % 4) * 32) >> 4;
-        mma_bf16_ss_w(tmem_s, dq + off, dk + off, idesc, kk > 0 ? 1u : 0u, leader);
+        if (FP8)
+            mma_f8_ss_w(tmem_s, dq + off, dk + off, idesc, kk > 0 ? 1u : 0u, leader);
+        else
+            mma_bf16_ss_w(tmem_s, dq + off, dk + off, idesc, kk > 0 ? 1u : 0u, leader);
     }
 }
 
-template <int D>
+template <int D, bool FP8>
 __device__ __forceinline__ void fwd_issue_pv(uint32_t tmem_o, uint32_t tmem_p, uint64_t dv,
                                              bool accumulate, int half, uint32_t leader) {
-    constexpr uint32_t idesc = idesc_bf16_f32(128, D, true);
+    using T = FwdTraits<D, FP8>;
+    constexpr uint32_t idesc = FP8 ? idesc_e4m3_f32(128, D, true) : idesc_bf16_f32(128, D, true);
+    constexpr int kHalfSteps = T::kPvSteps / 2;
 #pragma unroll
-    for (int kk = 4 * half; kk < 4 * half + 4; ++kk) {
-        // P: 16 keys = 8 TMEM columns of bf16 pairs. V: 16 keys = 2 swizzle
-        // atoms of 8 rows (2048 bytes); the 64-column panels are kPanelBytes
-        // apart (the descriptor's leading-dimension offset).
-        mma_bf16_ts_w(tmem_o, tmem_p + kk * 8, dv + ((kk * 2048) >> 4), idesc,
-                      (accumulate || kk > 0) ? 1u : 0u, leader);
+    for (int kk = kHalfSteps * half; kk < kHalfSteps * (half + 1); ++kk) {
+        // P: 8 TMEM columns per MMA (16 keys as bf16 pairs, or 32 keys as
+        // e4m3 quads). V: the same keys' rows, 8-row swizzle atoms of 1024
+        // bytes; bf16 V's two 64-column panels are kPanelBytes apart (the
+        // descriptor's leading-dimension offset).
+        if (FP8)
+            mma_f8_ts_w(tmem_o, tmem_p + kk * 8, dv + ((kk * T::kPvRowBytes) >> 4), idesc,
+                        (accumulate || kk > 0) ? 1u : 0u, leader);
+        else
+            mma_bf16_ts_w(tmem_o, tmem_p + kk * 8, dv + ((kk * T::kPvRowBytes) >> 4), idesc,
+                          (accumulate || kk > 0) ? 1u : 0u, leader);
     }
 }
 
 // Run by the whole MMA warp with converged control flow; lane 0 issues.
-template <int D, bool CAUSAL>
+template <int D, bool CAUSAL, bool FP8>
 __device__ void fwd_mma(const FwdParams& p, uint32_t tbase, uint32_t sQ, uint32_t sKV,
-                        const FwdBars<FwdTraits<D>::kSlots>& b, uint32_t leader,
+                        const FwdBars<FwdTraits<D, FP8>::kSlots>& b, uint32_t leader,
                         volatile int* abort_flag) {
-    using T = FwdTraits<D>;
+    using T = FwdTraits<D, FP8>;
     constexpr uint64_t kTileStep = T::kTileBytes >> 4;
     const uint64_t dq0 = sdesc_sw128(sQ, 16, 1024);
     const uint64_t dk0 = sdesc_sw128(sKV, 16, 1024);                  // K-major K tile
@@ -339,7 +373,7 @@ __device__ void fwd_mma(const FwdParams& p, uint32_t tbase, uint32_t sQ, uint32_
             tc_fence_after_sync();
             for (int t = 0; t < 2; ++t)
                 if (x.n[t] > 0) {
-                    fwd_issue_s<D>(tbase + colS[t], dq0 + t * kTileStep, dk0 + kslot * kTileStep,
+                    fwd_issue_s<D, FP8>(tbase + colS[t], dq0 + t * kTileStep, dk0 + kslot * kTileStep,
                                    leader);
                     mma_commit_w(b.s_full(t), leader);
                     // Q_t's last use in this unit: let the producer refill it now
@@ -366,13 +400,13 @@ __device__ void fwd_mma(const FwdParams& p, uint32_t tbase, uint32_t sQ, uint32_
                             !role_wait(b.o_free(t), (o_use[t] - 1) & 1, abort_flag))
                             goto done;
                         tc_fence_after_sync();
-                        fwd_issue_pv<D>(tbase + colO[t], tbase + colS[t], dv0 + vslot * kTileStep,
+                        fwd_issue_pv<D, FP8>(tbase + colO[t], tbase + colS[t], dv0 + vslot * kTileStep,
                                         j > 0, 0, leader);
                         if (EATTN_SPLIT_P) {
                             if (!role_wait(b.p_hi(t), p_phase[t], abort_flag)) goto done;
                             tc_fence_after_sync();
                         }
-                        fwd_issue_pv<D>(tbase + colO[t], tbase + colS[t], dv0 + vslot * kTileStep,
+                        fwd_issue_pv<D, FP8>(tbase + colO[t], tbase + colS[t], dv0 + vslot * kTileStep,
                                         true, 1, leader);
                         p_phase[t] ^= 1;
                         if (j == x.n[t] - 1) mma_commit_w(b.o_final(t), leader);
@@ -383,7 +417,7 @@ __device__ void fwd_mma(const FwdParams& p, uint32_t tbase, uint32_t sQ, uint32_
                     }
                     if (t == 1) mma_commit_w(b.kv_empty(vslot), leader);
                     if (j + 1 < x.n[t]) {
-                        fwd_issue_s<D>(tbase + colS[t], dq0 + t * kTileStep,
+                        fwd_issue_s<D, FP8>(tbase + colS[t], dq0 + t * kTileStep,
                                        dk0 + kslot * kTileStep, leader);
                         mma_commit_w(b.s_full(t), leader);
                         if (j + 2 == x.n[t]) mma_commit_w(b.q_empty(t), leader);
@@ -411,10 +445,11 @@ done: {
 }
 
 // --------------------------------------------------------------- softmax --
-template <int D, bool CAUSAL>
-__device__ void fwd_softmax(const FwdParams& p, uint32_t tbase, const FwdBars<FwdTraits<D>::kSlots>& b, int warp,
-                            int lane, volatile int* abort_flag) {
-    using T = FwdTraits<D>;
+template <int D, bool CAUSAL, bool FP8>
+__device__ void fwd_softmax(const FwdParams& p, uint32_t tbase,
+                            const FwdBars<FwdTraits<D, FP8>::kSlots>& b, int warp, int lane,
+                            volatile int* abort_flag) {
+    using T = FwdTraits<D, FP8>;
     const int t = warp >> 2;                 // which Q tile
     const int quarter = warp & 3;            // TMEM lane quarter this warp may access
     const int r = quarter * 32 + lane;       // row within the tile = TMEM lane
@@ -424,11 +459,13 @@ __device__ void fwd_softmax(const FwdParams& p, uint32_t tbase, const FwdBars<Fw
     const uint32_t bar_s = b.s_full(t);
     const uint32_t bar_plo = b.p_lo(t), bar_phi = b.p_hi(t);
     const uint32_t bar_of = b.o_final(t), bar_ofree = b.o_free(t);
-    const float c2 = p.scale_log2;
     uint32_t s_phase = 0, o_use = 0;
 
     FWD_FOR_EACH_UNIT(u, p) {
         const FwdUnit x = fwd_unit<CAUSAL>(u, p);
+        // scores in log2 units; e4m3 inputs fold their Q and K factors in here
+        const float c2 = FP8 ? p.scale_log2 * p.q_descale[x.bh] * p.k_descale[x.bh]
+                             : p.scale_log2;
         const int n = x.n[t];
         // sequence lengths are at most 2^30, so row indices and limits fit in int
         const int qrow = x.qb * 256 + t * 128 + r;
@@ -463,18 +500,19 @@ __device__ void fwd_softmax(const FwdParams& p, uint32_t tbase, const FwdBars<Fw
                 mx3 = fmax3(mx3, __uint_as_float(sr[c + 6]), __uint_as_float(sr[c + 7]));
             }
             const float mxs = fmax3(mx0, mx1, fmaxf(mx2, mx3)) * c2;
-            const bool need = mxs > m_ref + 8.0f;
+            const bool need = mxs > m_ref + T::kLazy;
             const bool any_need = __any_sync(0xffffffffu, need);
             const float m_new = need ? mxs : m_ref;
             const float alpha = need ? fast_exp2(m_ref - m_new) : 1.0f;
             m_ref = m_new;
-            const float base = (m_ref == -INFINITY) ? 0.f : m_ref;
+            const float base = (m_ref == -INFINITY) ? 0.f : m_ref - T::kShift;
             const f32x2_t c2x2 = f2_pack(c2, c2);
             const f32x2_t nbx2 = f2_pack(-base, -base);
             f32x2_t lsum_a = f2_pack(0.f, 0.f), lsum_b = f2_pack(0.f, 0.f);
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
-                uint32_t pk[32];
+                uint32_t pk[FP8 ? 16 : 32];     // bf16 pairs or e4m3 quads
+                float e_prev0 = 0.f, e_prev1 = 0.f;
 #pragma unroll
                 for (int i = 0; i < 32; ++i) {
                     const int c = 64 * h + 2 * i;
@@ -484,13 +522,19 @@ __device__ void fwd_softmax(const FwdParams& p, uint32_t tbase, const FwdBars<Fw
                     if (kPolyEvery<D> > 0 &&
                                (i % (kPolyEvery<D> > 0 ? kPolyEvery<D> : 1)) == kPolyEvery<D> - 1) {
                         exp2_poly_pair(xv, e0, e1);
-                        pk[i] = pack_bf16x2(e0, e1);
                     } else {
                         float x0, x1;
                         f2_unpack(xv, x0, x1);
                         e0 = fast_exp2(x0);
                         e1 = fast_exp2(x1);
+                    }
+                    if constexpr (!FP8) {
                         pk[i] = pack_bf16x2(e0, e1);
+                    } else if (i & 1) {
+                        pk[i / 2] = pack_e4m3x4(e_prev0, e_prev1, e0, e1);
+                    } else {
+                        e_prev0 = e0;
+                        e_prev1 = e1;
                     }
                     if (i & 1)
                         lsum_b = f2_add(lsum_b, f2_pack(e0, e1));
@@ -512,7 +556,10 @@ __device__ void fwd_softmax(const FwdParams& p, uint32_t tbase, const FwdBars<Fw
                         tmem_st32(tO + c, orr);
                     }
                 }
-                tmem_st32(tS + 32 * h, pk);
+                if constexpr (FP8)
+                    tmem_st16(tS + 16 * h, pk);
+                else
+                    tmem_st32(tS + 32 * h, pk);
                 if (EATTN_SPLIT_P || h == 1) {
                     tmem_wait_st();
                     tc_fence_before_sync();
@@ -532,7 +579,7 @@ __device__ void fwd_softmax(const FwdParams& p, uint32_t tbase, const FwdBars<Fw
         if (n > 0) {
             if (!warp_wait(bar_of, o_use & 1, abort_flag)) return;
             tc_fence_after_sync();
-            const float inv = l > 0.f ? 1.0f / l : 0.f;
+            const float inv = l > 0.f ? (FP8 ? p.v_descale[x.bh] : 1.0f) / l : 0.f;
 #pragma unroll
             for (int c = 0; c < D; c += 32) {
                 uint32_t orr[32];
@@ -560,17 +607,17 @@ __device__ void fwd_softmax(const FwdParams& p, uint32_t tbase, const FwdBars<Fw
         }
         if (row_valid)
             p.lse[(size_t)x.bh * p.Nq + qrow] =
-                l > 0.f ? (m_ref + log2f(l)) * 0.69314718055994531f : -INFINITY;
+                l > 0.f ? (m_ref - T::kShift + log2f(l)) * 0.69314718055994531f : -INFINITY;
     }
 }
 
 // ---------------------------------------------------------------- kernel --
-template <int D, bool CAUSAL>
+template <int D, bool CAUSAL, bool FP8 = false>
 __global__ void __launch_bounds__(384, 1)
     attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
                           const __grid_constant__ CUtensorMap tm_k,
                           const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
-    using T = FwdTraits<D>;
+    using T = FwdTraits<D, FP8>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -620,14 +667,14 @@ __global__ void __launch_bounds__(384, 1)
 
     if (warp < 8) {
         regs_increase<T::kSoftmaxRegs>();
-        fwd_softmax<D, CAUSAL>(p, tbase, b, warp, lane, abort_flag);
+        fwd_softmax<D, CAUSAL, FP8>(p, tbase, b, warp, lane, abort_flag);
     } else {
         regs_decrease<T::kOtherRegs>();
         const bool issuer_thread = EATTN_WARP_ISSUE ? true : lane == 0;
         if (warp == 8 && issuer_thread)
-            fwd_producer<D, CAUSAL>(p, &tm_q, &tm_k, &tm_v, sQ, sKV, b, lane == 0, abort_flag);
+            fwd_producer<D, CAUSAL, FP8>(p, &tm_q, &tm_k, &tm_v, sQ, sKV, b, lane == 0, abort_flag);
         else if (warp == 9 && issuer_thread)
-            fwd_mma<D, CAUSAL>(p, tbase, sQ, sKV, b, lane == 0, abort_flag);
+            fwd_mma<D, CAUSAL, FP8>(p, tbase, sQ, sKV, b, lane == 0, abort_flag);
     }
 
     tc_fence_before_sync();

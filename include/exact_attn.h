@@ -79,6 +79,33 @@ attn_status_t attn_fwd(const void *q, const void *k, const void *v, void *o, flo
                        void *stream);
 
 /*
+ * Prefill forward on 8-bit inputs: the same O and LSE as attn_fwd for the
+ * values x = descale * code, with Q, K and V given as e4m3 codes (OCP FP8
+ * E4M3: 1 sign, 4 exponent bits with bias 7, 3 mantissa bits, no infinities,
+ * 0x7F/0xFF NaN) and one fp32 descale factor per (b, h) for each of them.
+ *
+ * Defines: the FP8 path the pages name for FlashAttention-3 ("Describe Flash
+ * Attention at a high level" (mantramindai), section "Versions";
+ * "How FlashAttention Speeds Up the Attention Layer" (hassanahmed.net), the
+ * FlashAttention-3 paragraph). The pages give no format or scaling; this
+ * library reads them as e4m3 inputs with per-head descale factors, both
+ * products on the 8-bit tensor-core path (kind::f8f6f4), and P rounded to e4m3
+ * for the P V product (O is accumulated in fp32 and returned as bf16).
+ *
+ *   q                 e4m3 [B, H, Nq, 128]    (read; one byte per element)
+ *   k, v              e4m3 [B, H, Nkv, 128]   (read)
+ *   q/k/v_descale     fp32 [B, H]             (read; device memory)
+ *   o                 bf16 [B, H, Nq, 128]    (written)
+ *   lse               fp32 [B, H, Nq]         (written; natural log, as attn_fwd)
+ *   d must be 128 (ATTN_ERR_UNSUPPORTED otherwise); causal, scale and the
+ *   size limits as attn_fwd; q, k, v, o 16-byte aligned, the rest 4-byte.
+ */
+attn_status_t attn_fwd_fp8(const void *q, const void *k, const void *v, const float *q_descale,
+                           const float *k_descale, const float *v_descale, void *o, float *lse,
+                           int B, int H, int Nq, int Nkv, int d, int causal, float scale,
+                           void *stream);
+
+/*
  * Split-KV decode, step 1: per-chunk partials for one query row per (b, h).
  *
  * Defines: the decode method of "Describe Flash Attention at a high level"

@@ -31,7 +31,7 @@ def test_header_declares_the_boundary():
     names = declared_functions()
     for want in ("attn_fwd", "attn_decode_partials", "attn_lse_merge", "attn_decode_splitkv",
                  "attn_decode_workspace_bytes", "attn_status", "attn_strerror",
-                 "attn_abi_version", "attn_bwd", "attn_bwd_workspace_bytes"):
+                 "attn_abi_version", "attn_bwd", "attn_bwd_workspace_bytes", "attn_fwd_fp8"):
         assert want in names
 
 
@@ -116,6 +116,26 @@ def test_bwd_rejects_bad_arguments_without_launching(ea):
     assert call(d=80) == ea.ATTN_ERR_UNSUPPORTED
     assert call(dk=p + 8) == ea.ATTN_ERR_ALIGNMENT
     assert call(ws=p + 16) == ea.ATTN_ERR_ALIGNMENT
+
+
+def test_fwd_fp8_rejects_bad_arguments_without_launching(ea):
+    L = ea.lib
+    p = 0x10000
+
+    def call(**kw):
+        a = dict(dict(q=p, k=p, v=p, qd=p, kd=p, vd=p, o=p, lse=p, B=1, H=2, Nq=300, Nkv=300,
+                      d=128, causal=1, scale=0.088), **kw)
+        return L.attn_fwd_fp8(a["q"], a["k"], a["v"], a["qd"], a["kd"], a["vd"], a["o"],
+                              a["lse"], a["B"], a["H"], a["Nq"], a["Nkv"], a["d"], a["causal"],
+                              a["scale"], None)
+
+    assert call(vd=None) == ea.ATTN_ERR_INVALID_ARG
+    assert call(Nq=0) == ea.ATTN_ERR_INVALID_ARG
+    assert call(causal=3) == ea.ATTN_ERR_INVALID_ARG
+    assert call(scale=-1.0) == ea.ATTN_ERR_INVALID_ARG
+    assert call(d=64) == ea.ATTN_ERR_UNSUPPORTED
+    assert call(k=p + 8) == ea.ATTN_ERR_ALIGNMENT
+    assert call(qd=p + 2) == ea.ATTN_ERR_ALIGNMENT
 
 
 def test_package_fails_loudly_without_the_library(tmp_path):

@@ -13,6 +13,9 @@ no extra flush is needed between steps.
 ``--workload prefill_8k_bwd`` (or another ``*_bwd``) times the backward pass
 (dQ, dK, dV) of that prefill workload instead, one attn_bwd call per step.
 
+``--workload prefill_8k_fp8`` times the forward pass on e4m3 inputs
+(attn_fwd_fp8) of that workload.
+
 ``--impl reference`` times the fp64 CPU oracle on a bounded sample of the same
 workloads instead (the reference arm); it never touches the GPU path.
 
@@ -170,6 +173,7 @@ KERNEL_SOURCES = {
     "attn_decode_partials": ("decode_sm100.cuh", "ptx_sm100.cuh"),
     "attn_lse_merge": ("decode_sm100.cuh",),
     "attn_bwd_sm100": ("bwd_sm100.cuh", "ptx_sm100.cuh", "tmem_wide.cuh"),
+    "attn_fwd_sm100_e4m3": ("fwd_sm100.cuh", "ptx_sm100.cuh", "tmem_wide.cuh"),
 }
 
 
@@ -404,6 +408,158 @@ def oracle_bwd_sample(w, budget_s):
             break
         n *= 2
     return {"flops": flops, "seconds": dt, "n": n, "cores": orc.num_threads()}
+
+
+def oracle_fp8_sample(w, budget_s):
+    """Time the oracle's 8-bit entry on leading square blocks of one head (a
+    causal head's first n rows see only its first n keys); n doubles until one
+    call takes a quarter of the budget."""
+    import oracle
+    from seeded_inputs import fp8_codes, make_qkv_fp8
+    orc = oracle.get()
+    q8, k8, v8, qd, kd, vd = make_qkv_fp8(1, 1, w.Nq, w.Nkv, w.d, w.seed)
+    n = 256
+    while True:
+        c = lambda t: fp8_codes(t[:, :, :n])
+        t0 = time.perf_counter()
+        orc.attn_fwd_fp8(c(q8), c(k8), c(v8), qd.numpy(), kd.numpy(), vd.numpy(), w.causal,
+                         w.scale)
+        dt = time.perf_counter() - t0
+        flops = 4.0 * w.d * (n * (n + 1) // 2 if w.causal else n * n)
+        if dt > budget_s / 4 or 2 * n > min(w.Nq, w.Nkv):
+            break
+        n *= 2
+    return {"flops": flops, "seconds": dt, "n": n, "cores": orc.num_threads()}
+
+
+def run_fp8(args):
+    """Forward pass on e4m3 inputs (attn_fwd_fp8) of a prefill workload: codes and
+    per-head descale factors drawn from the workload's seed; one call per step."""
+    import torch
+    import torch.distributed as dist
+
+    import exact_io_aware_70_b200 as ea
+    from exact_io_aware_70_b200.replicas import max_over_ranks, replica_workload
+    from seeded_inputs import make_qkv_fp8
+
+    ws, rank, local = dist_env()
+    torch.cuda.set_device(local)
+    if ws > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    dev = torch.device("cuda", local)
+    stream = torch.cuda.current_stream()
+    sp = stream.cuda_stream
+    L = ea.lib
+    w = _maybe_batch(WORKLOADS[args.workload[:-len("_fp8")]], args.batch)
+    wr = replica_workload(w, rank)
+    ins = make_qkv_fp8(w.B, w.H, w.Nq, w.Nkv, w.d, wr.seed, device="cuda")
+    o = torch.empty((w.B, w.H, w.Nq, w.d), dtype=torch.bfloat16, device=dev)
+    lse = torch.empty((w.B, w.H, w.Nq), dtype=torch.float32, device=dev)
+    args_c = tuple(t.data_ptr() for t in ins) + (o.data_ptr(), lse.data_ptr(), w.B, w.H, w.Nq,
+                                                 w.Nkv, w.d, int(w.causal), w.scale, sp)
+
+    def step():
+        rc = L.attn_fwd_fp8(*args_c)
+        if rc != 0:
+            raise RuntimeError(f"attn_fwd_fp8: {ea.attn_strerror(rc)}")
+
+    for _ in range(args.warmup):
+        step()
+    if ea.attn_status() != 0:
+        raise RuntimeError("device status reported an error during warm-up")
+    K = args.steps
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(K + 1)]
+    with ClockSampler(local) as clk:
+        if ws > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+        for s in range(K):
+            ev[s].record(stream)
+            step()
+        ev[K].record(stream)
+        torch.cuda.synchronize()
+        if ws > 1:
+            dist.barrier()
+    if ea.attn_status() != 0:
+        raise RuntimeError("device status reported an error in the timed region")
+    total_ms = ev[0].elapsed_time(ev[K])
+    call_ms = statistics.mean(ev[s].elapsed_time(ev[s + 1]) for s in range(K))
+
+    e2e = None
+    if not args.no_e2e:
+        hin = [t.cpu().pin_memory() for t in ins]
+        hout = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in (o, lse)]
+        h2d = sum(t.numel() * t.element_size() for t in hin)
+        d2h = sum(t.numel() * t.element_size() for t in hout)
+        q8, k8, v8, qd, kd, vd = ins
+
+        def e2e_step():
+            for dst, src in zip(ins, hin):
+                dst.copy_(src, non_blocking=True)
+            ea.attn_fwd_fp8(q8, k8, v8, qd, kd, vd, o, lse, w.causal, w.scale)
+            for dst, src in zip(hout, (o, lse)):
+                dst.copy_(src, non_blocking=True)
+
+        e2e_step()
+        torch.cuda.synchronize()
+        E = max(2, min(K, 3))
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(E):
+            e2e_step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        if ea.attn_status() != 0:
+            raise RuntimeError("device status reported an error in the e2e region")
+        e2e = {"value": None, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
+               "d2h_bytes_per_step": d2h, "ms_per_step": e0.elapsed_time(e1) / E, "steps": E,
+               "path": "pinned host -> copy -> attn_fwd_fp8 -> copy back, per step, CUDA events"}
+    vals = max_over_ranks([total_ms, call_ms] + ([e2e["ms_per_step"]] if e2e else []), device=dev)
+    total_ms, call_ms = vals[0], vals[1]
+    if e2e:
+        e2e["ms_per_step"] = vals[2]
+        e2e["value"] = ws * prefill_flops(w) / (vals[2] * 1e-3) / 1e12
+    if ws > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return 0
+    pk = peaks()
+    fp8_peak = 2.0 * pk["bf16_tflops"]
+    a = prefill_flops(w) / (call_ms * 1e-3) / 1e12
+    roof = {"kernel": "attn_fwd_sm100 (e4m3)", "bound": "tensor", "achieved": a,
+            "peak": fp8_peak, "unit": "TFLOP/s", "frac": a / fp8_peak,
+            "peak_note": "measured bf16 peak x 2 (nominal e4m3 / bf16 dense ratio)",
+            "frac_of_bf16_peak": a / pk["bf16_tflops"],
+            "traffic": recorded_traffic().get("attn_fwd_sm100_e4m3"),
+            "algorithmic_bytes": prefill_bytes(w) // 2 + w.B * w.H * w.Nq * w.d,
+            "algorithmic_flops": prefill_flops(w), "ms": call_ms}
+    line = {
+        "metric": "attn fwd (e4m3 inputs) TFLOP/s & % FP8 tensor peak",
+        "value": ws * a, "unit": "TFLOP/s", "n_gpus": ws, "steps": K, "warmup": args.warmup,
+        "ms_per_step": total_ms / K, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "e4m3", "data": "synthetic",
+        "config": {"workload": args.workload, "B": w.B, "H": w.H, "N": w.Nq, "d": w.d,
+                   "causal": w.causal, "flop_per_step": prefill_flops(w),
+                   "l2": "inputs larger than L2 (126 MB); no flush" if not args.batch else
+                         "reduced batch for profiling",
+                   "parallelism": f"replicas x{ws}" if ws > 1 else "1 GPU"},
+        "roofline": roof,
+        "peaks": dict(pk, note="of measured" if pk["source"] == "measured" else "of fallback"),
+        "clocks": clk.summary(max_mhz_default=1965.0),
+        "gpu_launches": K, "e2e": e2e,
+    }
+    if ws == 1 and not args.no_cpu_baseline:
+        cb = oracle_fp8_sample(w, args.cpu_budget)
+        line["cpu_baseline"] = {
+            "value": cb["flops"] / cb["seconds"] / 1e12, "unit": "TFLOP/s", "cores": cb["cores"],
+            "kind": "oracle",
+            "sample": f"fp64 oracle on the decoded e4m3 inputs of the leading {cb['n']}x{cb['n']} "
+                      f"block of one head ({cb['flops'] / 1e9:.1f} GFLOP in {cb['seconds']:.2f} s)"}
+    print(json.dumps(line), flush=True)
+    return 0
 
 
 def run_bwd(args):
@@ -821,9 +977,10 @@ def main():
     ap.add_argument("--workload", default="step",
                     choices=["step", "prefill_8k", "prefill_16k", "gpt2_1k", "tiny", "decode_32k",
                              "decode_32k_paged", "prefill_8k_bwd", "prefill_16k_bwd",
-                             "gpt2_1k_bwd"],
+                             "gpt2_1k_bwd", "prefill_8k_fp8", "prefill_16k_fp8"],
                     help="step = prefill_8k + decode_32k (the default bench line); "
-                         "*_bwd = the backward pass of that prefill workload")
+                         "*_bwd = the backward pass of that prefill workload; "
+                         "*_fp8 = its forward pass on e4m3 inputs")
     ap.add_argument("--batch", type=int, default=0,
                     help="override the batch size (small profiling captures only)")
     ap.add_argument("--no-e2e", action="store_true")
@@ -839,6 +996,8 @@ def main():
         return run_reference(args)
     if args.workload.endswith("_bwd"):
         return run_bwd(args)
+    if args.workload.endswith("_fp8"):
+        return run_fp8(args)
     return run_ours(args)
 
 

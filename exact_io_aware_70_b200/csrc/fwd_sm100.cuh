@@ -41,7 +41,7 @@
 //   * Exponentials are base 2 with log2(e) folded into the scale, computed
 //     with MUFU ex2 on pairs prepared by sm_100's packed f32x2 FMA; the row
 //     max uses the three-input max. A fraction of the pairs can instead be
-//     exponentiated on the FMA pipe (exp2_poly_pair, kPolyEvery<D>); measured
+//     exponentiated on the FMA pipe (exp2_poly_pair, kPolyEvery<D, FP8>); measured
 //     on B200 it is slower at every fraction tried, at d=128 (MUFU and tensor
 //     core need the same cycles per step) and at d=64 (short sequences are
 //     latency-bound), so it is off by default. A masked
@@ -144,7 +144,7 @@ struct FwdTraits {
     static constexpr uint32_t kColO0 = 256, kColO1 = 256 + D;
 };
 
-// One exponent pair in every kPolyEvery<D> goes to the FMA-pipe polynomial
+// One exponent pair in every kPolyEvery<D, FP8> goes to the FMA-pipe polynomial
 // (0: none, the measured-best setting for both head dims).
 #ifndef EATTN_POLY_EVERY_D128
 #define EATTN_POLY_EVERY_D128 0
@@ -152,8 +152,16 @@ struct FwdTraits {
 #ifndef EATTN_POLY_EVERY_D64
 #define EATTN_POLY_EVERY_D64 0
 #endif
-template <int D>
-constexpr int kPolyEvery = (D == 128) ? EATTN_POLY_EVERY_D128 : EATTN_POLY_EVERY_D64;
+// e4m3 inputs halve the tensor-core time per tile while the exponentials stay,
+// so there the FMA-pipe polynomial has idle cycles to use: one pair in four
+// measured best on B200 (8K causal: 1158 -> 1289 TFLOP/s; one in 2, 3 and 6
+// in between).
+#ifndef EATTN_POLY_EVERY_FP8
+#define EATTN_POLY_EVERY_FP8 4
+#endif
+template <int D, bool FP8 = false>
+constexpr int kPolyEvery =
+    FP8 ? EATTN_POLY_EVERY_FP8 : ((D == 128) ? EATTN_POLY_EVERY_D128 : EATTN_POLY_EVERY_D64);
 
 // Unit handled by this CTA in round r (snake order), or -1 past the end.
 __device__ __forceinline__ int fwd_unit_of_round(int r, int num_units) {
@@ -519,8 +527,8 @@ __device__ void fwd_softmax(const FwdParams& p, uint32_t tbase,
                     const f32x2_t xv = f2_fma(
                         f2_pack(__uint_as_float(sr[c]), __uint_as_float(sr[c + 1])), c2x2, nbx2);
                     float e0, e1;
-                    if (kPolyEvery<D> > 0 &&
-                               (i % (kPolyEvery<D> > 0 ? kPolyEvery<D> : 1)) == kPolyEvery<D> - 1) {
+                    if (kPolyEvery<D, FP8> > 0 &&
+                               (i % (kPolyEvery<D, FP8> > 0 ? kPolyEvery<D, FP8> : 1)) == kPolyEvery<D, FP8> - 1) {
                         exp2_poly_pair(xv, e0, e1);
                     } else {
                         float x0, x1;

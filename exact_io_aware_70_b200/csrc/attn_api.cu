@@ -68,14 +68,15 @@ EncodeTiledFn get_encode_fn() {
 
 bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
-// Tensor map over a bf16 tensor viewed as [BH][N][D]; box = 128 rows x 64 columns,
-// 128-byte swizzle, out-of-range rows read as zero.
-bool encode_bf16_map(CUtensorMap* map, const void* base, int BH, int N, int D) {
+// Tensor map over a bf16 tensor viewed as [BH][N][D]; box = box_rows rows x 64
+// columns, 128-byte swizzle, out-of-range rows read as zero.
+bool encode_bf16_map(CUtensorMap* map, const void* base, int BH, int N, int D,
+                     int box_rows = 128) {
     EncodeTiledFn enc = get_encode_fn();
     if (!enc) return false;
     cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)N, (cuuint64_t)BH};
     cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)N * D * 2};
-    cuuint32_t box[3] = {64, 128, 1};
+    cuuint32_t box[3] = {64, (cuuint32_t)box_rows, 1};
     cuuint32_t estr[3] = {1, 1, 1};
     CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims,
                      strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
@@ -159,10 +160,11 @@ attn_status_t launch_bwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUt
             di.bwd_attr_set[slot] = true;
         }
     }
-    const long long rows = (long long)p.BH * p.Nq;
+    const long long prows = (long long)p.BH * p.NqPad;
     constexpr int kRowsPerBlock = 256 / (D / 8);
     attn_bwd_preprocess_kernel<D>
-        <<<(unsigned)((rows + kRowsPerBlock - 1) / kRowsPerBlock), 256, 0, stream>>>(p);
+        <<<(unsigned)((prows + kRowsPerBlock - 1) / kRowsPerBlock), 256, 0, stream>>>(p);
+    const long long rows = (long long)p.BH * p.Nq;
     // key blocks along x so that the CTAs resident at one time share a few
     // heads' Q and dO tiles in L2
     dim3 grid((p.Nkv + 127) / 128, p.BH);
@@ -439,8 +441,8 @@ attn_status_t attn_decode_splitkv(const void* q, const void* k, const void* v, v
 
 size_t attn_bwd_workspace_bytes(int B, int H, int Nq, int d) {
     if (B < 1 || H < 1 || Nq < 1 || (d != 64 && d != 128)) return 0;
-    const size_t rows = (size_t)B * H * Nq;
-    return (rows * 4 + 255) / 256 * 256 + rows * d * 4;
+    const size_t prow = (size_t)B * H * (((size_t)Nq + 63) / 64 * 64);
+    return 2 * ((prow * 4 + 255) / 256 * 256) + (size_t)B * H * Nq * d * 4;
 }
 
 attn_status_t attn_bwd(const void* q, const void* k, const void* v, const void* o,
@@ -463,16 +465,19 @@ attn_status_t attn_bwd(const void* q, const void* k, const void* v, const void* 
         !aligned(lse, 4) || !aligned(workspace, 256))
         return ATTN_ERR_ALIGNMENT;
     CUtensorMap tq, tk, tv, tdo;
-    if (!encode_bf16_map(&tq, q, BH, Nq, d) || !encode_bf16_map(&tk, k, BH, Nkv, d) ||
-        !encode_bf16_map(&tv, v, BH, Nkv, d) || !encode_bf16_map(&tdo, dout, BH, Nq, d))
+    if (!encode_bf16_map(&tq, q, BH, Nq, d, 64) || !encode_bf16_map(&tk, k, BH, Nkv, d) ||
+        !encode_bf16_map(&tv, v, BH, Nkv, d) || !encode_bf16_map(&tdo, dout, BH, Nq, d, 64))
         return ATTN_ERR_CUDA;
-    const size_t rows = (size_t)BH * Nq;
+    const int NqPad = (Nq + 63) / 64 * 64;
+    const size_t pbytes = ((size_t)BH * NqPad * 4 + 255) / 256 * 256;
     BwdParams p;
     p.o = static_cast<const uint16_t*>(o);
     p.dout = static_cast<const uint16_t*>(dout);
     p.lse = lse;
     p.delta = static_cast<float*>(workspace);
-    p.dq_acc = reinterpret_cast<float*>(static_cast<char*>(workspace) + (rows * 4 + 255) / 256 * 256);
+    p.lse2 = reinterpret_cast<float*>(static_cast<char*>(workspace) + pbytes);
+    p.dq_acc = reinterpret_cast<float*>(static_cast<char*>(workspace) + 2 * pbytes);
+    p.NqPad = NqPad;
     p.dq = static_cast<uint16_t*>(dq);
     p.dk = static_cast<uint16_t*>(dk);
     p.dv = static_cast<uint16_t*>(dv);

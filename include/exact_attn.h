@@ -227,9 +227,10 @@ attn_status_t attn_decode_splitkv_noalloc(const void *q, const void *k, const vo
 
 /*
  * Backward pass: bytes of device workspace attn_bwd needs, or 0 if the
- * arguments are invalid. Layout (owned by the caller, 256-byte aligned):
- * fp32 D [B, H, Nq] padded to 256 bytes, then the fp32 dQ accumulator
- * [B, H, Nq, d]. Nothing in it needs initialising.
+ * arguments are invalid. Layout (owned by the caller, 256-byte aligned), with
+ * NqPad = Nq rounded up to a multiple of 64: fp32 D [B, H, NqPad] and fp32
+ * LSE * log2(e) [B, H, NqPad], each padded to 256 bytes, then the fp32 dQ
+ * accumulator [B, H, Nq, d]. Nothing in it needs initialising.
  */
 size_t attn_bwd_workspace_bytes(int B, int H, int Nq, int d);
 
@@ -256,10 +257,10 @@ size_t attn_bwd_workspace_bytes(int B, int H, int Nq, int d);
  *               256-byte aligned; overwritten.
  *   d in {64, 128}; causal 0 or 1 (bottom-right, as attn_fwd); B * H <= 65535.
  *   A query row whose LSE is -inf (it sees no key) contributes nothing.
- *   Three kernels run on `stream` in order: D and zeroing of the accumulator,
- *   the main kernel (one CTA per 128-key block and head), and the dQ
- *   conversion. dQ is summed with fp32 atomic adds, so its last bits may vary
- *   from run to run; dK and dV do not.
+ *   Three kernels run on `stream` in order: D, LSE * log2(e) and zeroing of
+ *   the accumulator; the main kernel (one CTA per 128-key block and head,
+ *   64-row query blocks); and the dQ conversion. dQ is summed with fp32 atomic
+ *   adds, so its last bits may vary from run to run; dK and dV do not.
  */
 attn_status_t attn_bwd(const void *q, const void *k, const void *v, const void *o,
                        const void *dout, const float *lse, void *dq, void *dk, void *dv, int B,

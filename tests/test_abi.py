@@ -95,7 +95,7 @@ def test_bwd_rejects_bad_arguments_without_launching(ea):
     L = ea.lib
     p = 0x10000
     ws_need = ea.attn_bwd_workspace_bytes(1, 2, 300, 128)
-    assert ws_need == (2 * 300 * 4 + 255) // 256 * 256 + 2 * 300 * 128 * 4
+    assert ws_need == 2 * ((2 * 320 * 4 + 255) // 256 * 256) + 2 * 300 * 128 * 4
     assert ea.attn_bwd_workspace_bytes(1, 2, 300, 96) == 0
     assert ea.attn_bwd_workspace_bytes(1, 2, 0, 128) == 0
 

@@ -56,6 +56,11 @@
 //     released to the producer right after its last S product of the unit.
 //   * Tensor memory columns: S0 [0,128), S1 [128,256), O0 [256,256+d),
 //     O1 [256+d, 256+2d).
+//   * The same kernel serves e4m3 inputs (FP8 = true, head dim 128): 16 KB
+//     tiles of one 128-byte panel, an 8-slot K/V ring, both products as
+//     kind::f8f6f4 MMAs (K = 32), P rounded to e4m3 and packed four to a TMEM
+//     column, per-head descale factors folded into the exponent scale and the
+//     epilogue (see FwdTraits for the exponent shift that keeps P normal).
 #pragma once
 
 #include <cuda_bf16.h>

@@ -977,7 +977,7 @@ def main():
     ap.add_argument("--workload", default="step",
                     choices=["step", "prefill_8k", "prefill_16k", "gpt2_1k", "tiny", "decode_32k",
                              "decode_32k_paged", "prefill_8k_bwd", "prefill_16k_bwd",
-                             "gpt2_1k_bwd", "prefill_8k_fp8", "prefill_16k_fp8"],
+                             "gpt2_1k_bwd", "prefill_8k_fp8", "prefill_16k_fp8", "gpt2_1k_fp8"],
                     help="step = prefill_8k + decode_32k (the default bench line); "
                          "*_bwd = the backward pass of that prefill workload; "
                          "*_fp8 = its forward pass on e4m3 inputs")

@@ -126,8 +126,8 @@ def attn_fwd(q, k, v, o, lse, causal: bool, scale: float, stream=None) -> None:
 
 def attn_fwd_fp8(q, k, v, q_descale, k_descale, v_descale, o, lse, causal: bool, scale: float,
                  stream=None) -> None:
-    """O and LSE from e4m3 inputs. q [B,H,Nq,128], k/v [B,H,Nkv,128] torch.float8_e4m3fn;
-    *_descale [B,H] fp32; o [B,H,Nq,128] bf16; lse [B,H,Nq] fp32."""
+    """O and LSE from e4m3 inputs. q [B,H,Nq,d], k/v [B,H,Nkv,d] torch.float8_e4m3fn (d 64
+    or 128); *_descale [B,H] fp32; o [B,H,Nq,d] bf16; lse [B,H,Nq] fp32."""
     import torch
     B, H, Nq, d = q.shape
     Nkv = k.shape[2]

@@ -85,24 +85,26 @@ bool encode_bf16_map(CUtensorMap* map, const void* base, int BH, int N, int D,
     return r == CUDA_SUCCESS;
 }
 
-// Tensor map over an 8-bit tensor viewed as [BH][N][D] with D = 128: box =
-// 128 rows x 128 bytes, 128-byte swizzle, out-of-range rows read as zero.
+// Tensor map over an 8-bit tensor viewed as [BH][N][D] with D = 128 or 64: box =
+// 128 rows x D bytes, 128-byte swizzle (64-byte swizzle for D = 64), rows past
+// N read as zero.
 bool encode_u8_map(CUtensorMap* map, const void* base, int BH, int N, int D) {
     EncodeTiledFn enc = get_encode_fn();
     if (!enc) return false;
     cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)N, (cuuint64_t)BH};
     cuuint64_t strides[2] = {(cuuint64_t)D, (cuuint64_t)N * D};
-    cuuint32_t box[3] = {128, 128, 1};
+    cuuint32_t box[3] = {(cuuint32_t)D, 128, 1};
     cuuint32_t estr[3] = {1, 1, 1};
     CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(base), dims, strides,
-                     box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                     box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                     D == 64 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B,
                      CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS;
 }
 
 struct DeviceInfo {
     int sms = 0;
-    bool fwd_attr_set[6] = {false, false, false, false, false, false};
+    bool fwd_attr_set[8] = {false, false, false, false, false, false, false, false};
     bool bwd_attr_set[4] = {false, false, false, false};
 };
 DeviceInfo g_dev[64];
@@ -128,7 +130,7 @@ attn_status_t launch_fwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUt
         if (di.sms == 0 &&
             cudaDeviceGetAttribute(&di.sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
             return ATTN_ERR_CUDA;
-        const int slot = (FP8 ? 4 : (D == 128 ? 2 : 0)) + (CAUSAL ? 1 : 0);
+        const int slot = (FP8 ? 4 : 0) + (D == 128 ? 2 : 0) + (CAUSAL ? 1 : 0);
         if (!di.fwd_attr_set[slot]) {
             if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                      T::kSmemBytes) != cudaSuccess)
@@ -250,7 +252,7 @@ attn_status_t attn_fwd_fp8(const void* q, const void* k, const void* v, const fl
     if (!(scale > 0.f) || !std::isfinite(scale)) return ATTN_ERR_INVALID_ARG;
     attn_status_t s = check_sizes(B, H, Nq, Nkv);
     if (s != ATTN_OK) return s;
-    if (d != 128) return ATTN_ERR_UNSUPPORTED;
+    if (d != 64 && d != 128) return ATTN_ERR_UNSUPPORTED;
     if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) ||
         !aligned(lse, 4) || !aligned(q_descale, 4) || !aligned(k_descale, 4) ||
         !aligned(v_descale, 4))
@@ -275,8 +277,11 @@ attn_status_t attn_fwd_fp8(const void* q, const void* k, const void* v, const fl
     p.num_units = (int)units;
     p.scale_log2 = scale * kLog2e;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    return causal ? launch_fwd<128, true, true>(tq, tk, tv, p, st)
-                  : launch_fwd<128, false, true>(tq, tk, tv, p, st);
+    if (d == 128)
+        return causal ? launch_fwd<128, true, true>(tq, tk, tv, p, st)
+                      : launch_fwd<128, false, true>(tq, tk, tv, p, st);
+    return causal ? launch_fwd<64, true, true>(tq, tk, tv, p, st)
+                  : launch_fwd<64, false, true>(tq, tk, tv, p, st);
 }
 
 attn_status_t attn_decode_partials(const void* q, const void* k, const void* v, float* o_part,

@@ -107,20 +107,25 @@ struct FwdParams {
 
 // FP8 = true: Q, K, V are e4m3 codes with per-(batch*head) descale factors;
 // S and P V run as tcgen05.mma kind::f8f6f4 (K = 32 per instruction), P is
-// rounded to e4m3 in tensor memory. Head dim 128 only (a 128-byte row).
+// rounded to e4m3 in tensor memory. At head dim 64 an e4m3 row is 64 bytes,
+// so those tiles use the 64-byte swizzle (8-row atoms of 512 bytes).
 template <int D, bool FP8 = false>
 struct FwdTraits {
     static_assert(D == 64 || D == 128, "head dim 64 or 128");
-    static_assert(!FP8 || D == 128, "e4m3 inputs: head dim 128");
     static constexpr int kElemBytes = FP8 ? 1 : 2;
     static constexpr int kRows = 128;                     // rows of a Q, K or V tile
-    static constexpr int kPanelBytes = 128 * 128;         // 128 rows x 128 bytes (one swizzle panel)
-    static constexpr int kPanelElems = 128 / kElemBytes;  // elements of a row in one panel
-    static constexpr int kPanels = D * kElemBytes / 128;
+    // bytes of one row within a swizzle panel: 128 (128-byte swizzle), or 64
+    // for e4m3 at head dim 64 (64-byte swizzle)
+    static constexpr int kRowBytes = D * kElemBytes < 128 ? D * kElemBytes : 128;
+    static constexpr bool kSwizzle64 = kRowBytes == 64;
+    static constexpr int kAtomBytes = 8 * kRowBytes;      // 8-row swizzle atom (descriptor SBO)
+    static constexpr int kPanelBytes = 128 * kRowBytes;   // 128 rows of one swizzle panel
+    static constexpr int kPanelElems = kRowBytes / kElemBytes;  // elements of a row in one panel
+    static constexpr int kPanels = D * kElemBytes / kRowBytes;
     static constexpr int kTileBytes = kPanels * kPanelBytes;
     static constexpr int kKSteps = D * kElemBytes / 32;   // 32-byte K steps of S = Q K^T
     static constexpr int kPvSteps = FP8 ? 4 : 8;          // MMAs of P V per 128 keys
-    static constexpr int kPvRowBytes = FP8 ? 4096 : 2048; // V bytes one P V MMA consumes
+    static constexpr int kPvRowBytes = (FP8 ? 32 : 16) * kRowBytes;   // V bytes one P V MMA consumes
     // e4m3 P: exponents are taken against (reference max - kShift), so a row's
     // largest values of P lie in [2^6, 2^8] and e4m3's subnormal range (below
     // 2^-6) only holds values under 2^-12 of the row maximum; the lazy-rescale
@@ -128,7 +133,8 @@ struct FwdTraits {
     // The shift cancels in O = acc / l and is taken out of the LSE.
     static constexpr float kShift = FP8 ? 6.0f : 0.0f;
     static constexpr float kLazy = FP8 ? 2.0f : 8.0f;
-    static constexpr int kSlots = FP8 ? 8 : ((D == 128) ? EATTN_KV_SLOTS_D128 : 8);   // K/V ring depth
+    static constexpr int kSlots =
+        FP8 ? (D == 128 ? 8 : 16) : ((D == 128) ? EATTN_KV_SLOTS_D128 : 8);   // K/V ring depth
     static_assert(kSlots >= 2, "the ring holds K_j and V_j at once");
     static_assert(!EATTN_KV_PAIR_BARRIER || kSlots % 2 == 0, "K/V pairs need an even ring");
     static constexpr int kThreads = 384;                  // 3 warpgroups
@@ -320,6 +326,15 @@ fail: {
 }
 
 // ------------------------------------------------------------ MMA issuer --
+// Shared-memory descriptor of a tile in the traits' swizzle: 128-byte (layout
+// type 2, 1024-byte atoms) or 64-byte (layout type 4, 512-byte atoms).
+template <class T>
+__device__ __forceinline__ uint64_t fwd_sdesc(uint32_t saddr, uint32_t lbo_bytes) {
+    uint64_t d = sdesc_sw128(saddr, lbo_bytes, T::kAtomBytes);
+    if (T::kSwizzle64) d = (d & ~(uint64_t(7) << 61)) | (uint64_t(4) << 61);
+    return d;
+}
+
 // Descriptor bases are computed once; an operand at byte offset `off` from a
 // base is the base plus off >> 4 (the start-address field never overflows:
 // shared memory addresses are below 2^18).
@@ -368,9 +383,9 @@ __device__ void fwd_mma(const FwdParams& p, uint32_t tbase, uint32_t sQ, uint32_
                         volatile int* abort_flag) {
     using T = FwdTraits<D, FP8>;
     constexpr uint64_t kTileStep = T::kTileBytes >> 4;
-    const uint64_t dq0 = sdesc_sw128(sQ, 16, 1024);
-    const uint64_t dk0 = sdesc_sw128(sKV, 16, 1024);                  // K-major K tile
-    const uint64_t dv0 = sdesc_sw128(sKV, T::kPanelBytes, 1024);      // MN-major V tile
+    const uint64_t dq0 = fwd_sdesc<T>(sQ, 16);
+    const uint64_t dk0 = fwd_sdesc<T>(sKV, 16);                       // K-major K tile
+    const uint64_t dv0 = fwd_sdesc<T>(sKV, T::kPanelBytes);           // MN-major V tile
     const uint32_t colS[2] = {T::kColS0, T::kColS1};
     const uint32_t colO[2] = {T::kColO0, T::kColO1};
     uint32_t kv_iter = 0, q_use = 0;

@@ -92,12 +92,12 @@ attn_status_t attn_fwd(const void *q, const void *k, const void *v, void *o, flo
  * products on the 8-bit tensor-core path (kind::f8f6f4), and P rounded to e4m3
  * for the P V product (O is accumulated in fp32 and returned as bf16).
  *
- *   q                 e4m3 [B, H, Nq, 128]    (read; one byte per element)
- *   k, v              e4m3 [B, H, Nkv, 128]   (read)
- *   q/k/v_descale     fp32 [B, H]             (read; device memory)
- *   o                 bf16 [B, H, Nq, 128]    (written)
+ *   q                 e4m3 [B, H, Nq, d]      (read; one byte per element)
+ *   k, v              e4m3 [B, H, Nkv, d]     (read)
+ *   q/k/v_descale     fp32 [B, H]             (read; device memory; finite)
+ *   o                 bf16 [B, H, Nq, d]      (written)
  *   lse               fp32 [B, H, Nq]         (written; natural log, as attn_fwd)
- *   d must be 128 (ATTN_ERR_UNSUPPORTED otherwise); causal, scale and the
+ *   d in {64, 128} (ATTN_ERR_UNSUPPORTED otherwise); causal, scale and the
  *   size limits as attn_fwd; q, k, v, o 16-byte aligned, the rest 4-byte.
  */
 attn_status_t attn_fwd_fp8(const void *q, const void *k, const void *v, const float *q_descale,

@@ -133,7 +133,7 @@ def test_fwd_fp8_rejects_bad_arguments_without_launching(ea):
     assert call(Nq=0) == ea.ATTN_ERR_INVALID_ARG
     assert call(causal=3) == ea.ATTN_ERR_INVALID_ARG
     assert call(scale=-1.0) == ea.ATTN_ERR_INVALID_ARG
-    assert call(d=64) == ea.ATTN_ERR_UNSUPPORTED
+    assert call(d=96) == ea.ATTN_ERR_UNSUPPORTED
     assert call(k=p + 8) == ea.ATTN_ERR_ALIGNMENT
     assert call(qd=p + 2) == ea.ATTN_ERR_ALIGNMENT
 

@@ -75,8 +75,7 @@ def check_head(o_gpu, lse_gpu, q8, k8, v8, qd, kd, vd, causal, scale, what):
     return float((err / np.where(allowed > 0, allowed, 1.0)).max())
 
 
-def _parity(B, H, Nq, Nkv, causal, seed):
-    d = 128
+def _parity(B, H, Nq, Nkv, causal, seed, d=128):
     scale = float(np.float32(1.0 / np.sqrt(d)))
     q8, k8, v8, qd, kd, vd = make_qkv_fp8(B, H, Nq, Nkv, d, seed)
     o, lse = run_fp8(*(t.cuda() for t in (q8, k8, v8, qd, kd, vd)), causal, scale)
@@ -87,6 +86,7 @@ def _parity(B, H, Nq, Nkv, causal, seed):
                        vd[b, h], causal, scale, f"fp8 B{B} H{H} {Nq}x{Nkv} causal{int(causal)} ({b},{h})")
 
 
+@pytest.mark.parametrize("d", [128, 64])
 @pytest.mark.parametrize("B,H,Nq,Nkv,causal", [
     (1, 1, 128, 128, False),
     (1, 1, 128, 128, True),
@@ -97,8 +97,14 @@ def _parity(B, H, Nq, Nkv, causal, seed):
     (1, 1, 1, 1, False),
     (1, 3, 2048, 2048, True),     # many K/V tiles per row: lazy rescaling and ring wrap
 ])
-def test_fp8_matches_oracle(B, H, Nq, Nkv, causal):
-    _parity(B, H, Nq, Nkv, causal, seed=Nq * 5 + Nkv + int(causal))
+def test_fp8_matches_oracle(B, H, Nq, Nkv, causal, d):
+    _parity(B, H, Nq, Nkv, causal, seed=Nq * 5 + Nkv + int(causal) + d, d=d)
+
+
+def test_fp8_gpt2_1k_full():
+    """The GPT-2-style workload (B=8, H=12, N=1024, d=64, causal) in e4m3, every head."""
+    w = WORKLOADS["gpt2_1k"]
+    _parity(w.B, w.H, w.Nq, w.Nkv, w.causal, w.seed, d=w.d)
 
 
 def test_fp8_prefill_8k_one_head():
@@ -112,10 +118,10 @@ def test_fp8_prefill_8k_one_head():
                w.causal, w.scale, "fp8 prefill_8k head 9")
 
 
-def test_fp8_rejects_head_dim_64():
+def test_fp8_rejects_head_dim_96():
     m = gpu_util.ea()
-    q8, k8, v8, qd, kd, vd = (t.cuda() for t in make_qkv_fp8(1, 1, 128, 128, 64, 1))
-    o = torch.empty((1, 1, 128, 64), dtype=torch.bfloat16, device="cuda")
+    q8, k8, v8, qd, kd, vd = (t.cuda() for t in make_qkv_fp8(1, 1, 128, 128, 96, 1))
+    o = torch.empty((1, 1, 128, 96), dtype=torch.bfloat16, device="cuda")
     lse = torch.empty((1, 1, 128), dtype=torch.float32, device="cuda")
     with pytest.raises(m.AttnError):
         m.attn_fwd_fp8(q8, k8, v8, qd, kd, vd, o, lse, False, 0.125)

@@ -178,11 +178,17 @@ KERNEL_SOURCES = {
 
 
 def kernel_source_hash(kernel):
+    """Hash of the kernel's device sources with // comments and blank lines
+    dropped, so that editing a comment does not retire a recorded figure."""
+    import re
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "exact_io_aware_70_b200", "csrc")
     for f in KERNEL_SOURCES[kernel]:
-        with open(os.path.join(csrc, f), "rb") as fh:
-            h.update(fh.read())
+        with open(os.path.join(csrc, f), encoding="utf-8") as fh:
+            for line in fh:
+                code = re.sub(r"//.*", "", line).rstrip()
+                if code:
+                    h.update(code.encode() + b"\n")
     return h.hexdigest()[:16]
 
 

@@ -25,7 +25,7 @@
 //     descriptors precomputed per tile and advanced by constant offsets. A
 //     tcgen05.mma costs the issuing thread about 48 cycles (measured), close
 //     to the 64 cycles one 128x128x16 MMA keeps the tensor core busy, so this
-//     thread's loop is kept as short as possible.: S_t = Q_t K_j^T into
+//     thread's loop is kept as short as possible: S_t = Q_t K_j^T into
 //     tensor memory (fp32, 128x128), and O_t += P_t V_j with P_t read straight
 //     from tensor memory (bf16, aliased over S_t's first 64 columns).
 //   * 384 threads = 3 warpgroups; warps 10-11 only complete the third
@@ -41,10 +41,11 @@
 //   * Exponentials are base 2 with log2(e) folded into the scale, computed
 //     with MUFU ex2 on pairs prepared by sm_100's packed f32x2 FMA; the row
 //     max uses the three-input max. A fraction of the pairs can instead be
-//     exponentiated on the FMA pipe (exp2_poly_pair, kPolyEvery<D, FP8>); measured
-//     on B200 it is slower at every fraction tried, at d=128 (MUFU and tensor
-//     core need the same cycles per step) and at d=64 (short sequences are
-//     latency-bound), so it is off by default. A masked
+//     exponentiated on the FMA pipe (exp2_poly_pair, kPolyEvery<D, FP8>). For
+//     bf16 inputs it is slower at every fraction tried (the MMA pipe, not the
+//     exponentials, sets the pace: a copy of the kernel without exponentials
+//     runs at the same speed), so it is off; for e4m3 inputs, whose products
+//     take half the tensor cycles, one pair in four is faster. A masked
 //     (-inf) score comes out of the polynomial as about 2^-125 rather than 0:
 //     negligible next to the row sum (at least 1 once a row has seen a
 //     visible key), and rows with
@@ -56,8 +57,9 @@
 //     released to the producer right after its last S product of the unit.
 //   * Tensor memory columns: S0 [0,128), S1 [128,256), O0 [256,256+d),
 //     O1 [256+d, 256+2d).
-//   * The same kernel serves e4m3 inputs (FP8 = true, head dim 128): 16 KB
-//     tiles of one 128-byte panel, an 8-slot K/V ring, both products as
+//   * The same kernel serves e4m3 inputs (FP8 = true): tiles of one swizzle
+//     panel (16 KB of 128-byte rows at d=128, an 8-slot K/V ring; 8 KB of
+//     64-byte rows with the 64-byte swizzle at d=64, 16 slots), both products as
 //     kind::f8f6f4 MMAs (K = 32), P rounded to e4m3 and packed four to a TMEM
 //     column, per-head descale factors folded into the exponent scale and the
 //     epilogue (see FwdTraits for the exponent shift that keeps P normal).

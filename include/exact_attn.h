@@ -16,7 +16,8 @@
  *     never allocates, frees or keeps them past the call.
  *   - Tensors are dense and row-major: Q, O are [B, H, Nq, d]; K, V are
  *     [B, H, Nkv, d]; LSE is [B, H, Nq]. Q, K, V, O are bfloat16 (passed as
- *     void*); LSE and split partials are fp32.
+ *     void*) except where an entry point says otherwise (attn_fwd_fp8 reads
+ *     e4m3 Q, K, V); LSE, split partials and workspaces are fp32.
  *   - Every call is asynchronous on `stream` (a cudaStream_t passed as void*;
  *     NULL means the legacy default stream). It returns after enqueueing.
  *   - Argument errors are reported synchronously, before anything is launched:
@@ -270,8 +271,9 @@ attn_status_t attn_bwd(const void *q, const void *k, const void *v, const void *
 /*
  * Synchronises `stream`, then returns and clears the device status word:
  * ATTN_ERR_TIMEOUT if a kernel's pipeline wait gave up since the last call
- * (its outputs are then invalid), ATTN_ERR_CUDA if the stream reported an
- * error, ATTN_OK otherwise.
+ * (its outputs are then invalid), ATTN_ERR_BAD_INDEX if a paged decode met an
+ * out-of-range block-table entry or length (those keys were skipped),
+ * ATTN_ERR_CUDA if the stream reported an error, ATTN_OK otherwise.
  */
 attn_status_t attn_status(void *stream);
 

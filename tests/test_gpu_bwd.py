@@ -70,9 +70,20 @@ def _parity(B, H, Nq, Nkv, d, causal, seed):
     (1, 1, 1, 1, 64, False),          # single element
     (1, 1, 1, 300, 128, True),        # one query row: sees every key
     (2, 3, 640, 640, 64, False),
+    (1, 2, 2048, 2048, 128, False),   # long non-causal: 32 query steps per key block
+    (1, 1, 1500, 4000, 64, True),     # Nq < Nkv at length
 ])
 def test_bwd_matches_oracle(B, H, Nq, Nkv, d, causal):
     _parity(B, H, Nq, Nkv, d, causal, seed=Nq * 7 + Nkv + d + int(causal))
+
+
+def test_bwd_other_scale():
+    """scale 0.5 on d = 128 (sharper softmax): the gradients through the error model."""
+    B, H, N, d = 1, 2, 600, 128
+    q, k, v = (t.cuda() for t in make_qkv(B, H, N, N, d, 91))
+    do = make_dout(B, H, N, d, 91, device="cuda")
+    dq, dk, dv, o = run_bwd(q, k, v, do, True, 0.5)
+    check_heads(q, k, v, do, o, dq, dk, dv, True, 0.5, [(0, 0), (0, 1)], "scale 0.5")
 
 
 def test_bwd_gpt2_1k_full():

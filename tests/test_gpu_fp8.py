@@ -101,6 +101,10 @@ def test_fp8_matches_oracle(B, H, Nq, Nkv, causal, d):
     _parity(B, H, Nq, Nkv, causal, seed=Nq * 5 + Nkv + int(causal) + d, d=d)
 
 
+def test_fp8_long_noncausal_d64():
+    _parity(1, 1, 4096, 4096, False, 55, d=64)
+
+
 def test_fp8_gpt2_1k_full():
     """The GPT-2-style workload (B=8, H=12, N=1024, d=64, causal) in e4m3, every head."""
     w = WORKLOADS["gpt2_1k"]

@@ -57,34 +57,38 @@ def build(force: bool = False, verbose: bool = False) -> str:
 # Fewer at launch would make the softmax warpgroups' increase wait forever, so
 # the build refuses to produce such a library.
 FWD_LAUNCH_REGS = 168
-# The backward kernel runs 14 warps per CTA; registers are split between the
-# SM's four schedulers, so four warps on one scheduler cap a thread at 128
-# registers. More would make every launch fail ("too many resources").
-BWD_MAX_REGS = 128
+# The backward kernel launches 20 warps with this many registers each and
+# redistributes them with setmaxnreg (BwdTraits::kLaunchRegs); with fewer at
+# launch the P/dS warpgroups' increase would wait forever, and more would not
+# fit five warps per SM scheduler, so the build requires exactly this count.
+BWD_LAUNCH_REGS = 96
 
 
 def check_register_budget(ptxas_log: str) -> None:
     current = None
     seen = 0
+    seen_bwd = 0
     for line in ptxas_log.splitlines():
         m = re.search(r"Compiling entry function '([^']+)'", line)
         if m:
             current = m.group(1)
             continue
         m = re.search(r"Used (\d+) registers", line)
-        if m and current and "attn_bwd_sm100_kernel" in current and int(m.group(1)) > BWD_MAX_REGS:
-            os.remove(LIB)
-            raise RuntimeError(f"{current} uses {m.group(1)} registers, more than "
-                               f"{BWD_MAX_REGS}: its 448-thread launch would fail")
+        if m and current and "attn_bwd_sm100_kernel" in current:
+            seen_bwd += 1
+            if int(m.group(1)) != BWD_LAUNCH_REGS:
+                os.remove(LIB)
+                raise RuntimeError(f"{current} uses {m.group(1)} registers, expected "
+                                   f"{BWD_LAUNCH_REGS}: the setmaxnreg split would not fit")
         if m and current and "attn_fwd_sm100_kernel" in current:
             seen += 1
             if int(m.group(1)) != FWD_LAUNCH_REGS:
                 os.remove(LIB)
                 raise RuntimeError(f"{current} uses {m.group(1)} registers, expected "
                                    f"{FWD_LAUNCH_REGS}: the setmaxnreg split would not fit")
-    if seen == 0:
+    if seen == 0 or seen_bwd == 0:
         os.remove(LIB)
-        raise RuntimeError("ptxas register report for the prefill kernel not found")
+        raise RuntimeError("ptxas register report for the prefill or backward kernel not found")
 
 
 if __name__ == "__main__":

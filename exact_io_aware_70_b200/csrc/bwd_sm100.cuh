@@ -20,8 +20,8 @@
 //      queries), so that one thread owns one key row of P^T and dS^T and both
 //      can stay in tensor memory as the A operand of dV += P^T dO_i and
 //      dK += dS^T Q_i. dS^T also goes to shared memory as the B operand of
-//      dQ_i^T = K_j^T dS^T (M = head dim), whose rows a reduction warpgroup
-//      adds into the fp32 dQ accumulator, 128 contiguous bytes per
+//      dQ_i^T = K_j^T dS^T (M = head dim), whose rows two reduction warpgroups
+//      add into the fp32 dQ accumulator, 128 contiguous bytes per
 //      instruction. Two tensor-memory stages let the tensor core work on one
 //      query block while the P/dS warps work on the next.
 //   3. attn_bwd_postprocess: dQ = bf16(scale * accumulator).
@@ -114,9 +114,21 @@ struct BwdTraits {
     static constexpr int kStages = 3;                   // Q_i, dO_i, LSE/D ring depth
     static constexpr int kLDBytes = 2 * kQRows * 4;     // LSE*log2e and D of 64 rows
     static constexpr int kDSBytes = 128 * kQRows * 2;   // dS^T: 128 keys x 64 queries bf16
-    static constexpr int kThreads = 448;  // warps 0-7 P/dS, 8-11 dQ reduction, 12 TMA, 13 MMA
+    // warps 0-7 P/dS, 8-15 dQ reduction (8-11 query columns 0-31 of a step,
+    // 12-15 columns 32-63), 16 TMA, 17 MMA, 18-19 idle
+    static constexpr int kThreads = 640;
     static constexpr int kComputeThreads = 256;
-    static constexpr int kReduceThreads = 128;
+    static constexpr int kReduceThreads = 256;
+    // Registers: the launch gives every thread kLaunchRegs (the build checks
+    // that ptxas gave the kernel exactly that many); setmaxnreg then moves them
+    // to the P/dS warpgroups. The split must fit the launch's total, and per
+    // SM scheduler (warps w, w+4, w+8, w+12, w+16) the 16384-register file.
+    static constexpr int kLaunchRegs = 96;
+    static constexpr int kPdsRegs = 120, kRedRegs = 80, kOtherRegs = 72;
+    static_assert(256 * kPdsRegs + 256 * kRedRegs + 128 * kOtherRegs <= kThreads * kLaunchRegs,
+                  "register split exceeds the launch allocation");
+    static_assert((2 * kPdsRegs + 2 * kRedRegs + kOtherRegs) * 32 <= 16384,
+                  "register split exceeds a scheduler's register file");
     static constexpr int kNumBars = 16;
     static constexpr int kSmemBytes = 1024 + 2 * kKTile + kStages * (2 * kQTile + kLDBytes) +
                                       2 * kDSBytes + kNumBars * 8 + 16;
@@ -161,7 +173,7 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
 }
 
 template <int D, bool CAUSAL>
-__global__ void __launch_bounds__(448, 1)
+__global__ void __launch_bounds__(640, 1)
     attn_bwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
                           const __grid_constant__ CUtensorMap tm_k,
                           const __grid_constant__ CUtensorMap tm_v,
@@ -207,7 +219,7 @@ __global__ void __launch_bounds__(448, 1)
         *abort_flag = 0;
         fence_mbar_init();
     }
-    if (warp == 13) {
+    if (warp == 17) {
         tmem_alloc(smem_addr(tmem_holder), T::kTmemCols);
         tmem_relinquish();
     }
@@ -216,7 +228,11 @@ __global__ void __launch_bounds__(448, 1)
     tc_fence_after_sync();
     const uint32_t tbase = *tmem_holder;
 
-    if (warp == 12) {
+    if (warp >= 16) regs_decrease<T::kOtherRegs>();
+    else if (warp >= 8) regs_decrease<T::kRedRegs>();
+    else regs_increase<T::kPdsRegs>();
+
+    if (warp == 16) {
         // ------------------------------------------------ TMA producer --
         if (lane == 0 && nsteps > 0) {
             int issued = 0;
@@ -254,7 +270,7 @@ __global__ void __launch_bounds__(448, 1)
                 if (cnt > 0) mbar_wait(b.qd_full(st), (cnt - 1) & 1, &no_abort, &g_attn_status);
             }
         }
-    } else if (warp == 13) {
+    } else if (warp == 17) {
         // -------------------------------------------------- MMA issuer --
         if (lane == 0 && nsteps > 0) {
             constexpr uint32_t id_s = idesc_bf16_f32(128, T::kQRows, false);   // A, B K-major
@@ -327,9 +343,10 @@ __global__ void __launch_bounds__(448, 1)
             volatile int no_abort = 0;
             mbar_wait(b.fin(), 0, &no_abort, &g_attn_status);
         }
-    } else if (warp >= 8) {
-        // ------------------------------- dQ reduction (warps 8-11, lane = head-dim index) --
-        const int quarter = warp - 8;
+    } else if (warp >= 8 && warp < 16) {
+        // ---------------- dQ reduction (warps 8-15, lane = head-dim index, 32 query columns) --
+        const int quarter = warp & 3;
+        const int cols = 32 * ((warp - 8) >> 2);   // this warp's first query column
         const int c = quarter * 32 + lane;
         const uint32_t lane_off = uint32_t(quarter * 32) << 16;
         float* dq_head = p.dq_acc + (size_t)bh * p.Nq * D + (c < D ? c : 0);
@@ -338,20 +355,26 @@ __global__ void __launch_bounds__(448, 1)
             bool ok = mbar_wait(b.dq_full(x), (s >> 1) & 1, abort_flag, &g_attn_status);
             if (!__all_sync(0xffffffffu, ok)) break;
             tc_fence_after_sync();
-            uint32_t v[64];
-            tmem_ld64(tbase + lane_off + T::col_stage(x), v);
-            tmem_wait_ld64(v);
+            uint32_t v[32];
+            tmem_ld32(tbase + lane_off + T::col_stage(x) + cols, v);
+            tmem_wait_ld(v);
             tc_fence_before_sync();
             mbar_arrive(b.dq_free(x));
-            const int row0 = (i0 + s) * T::kQRows;
+            const int row0 = (i0 + s) * T::kQRows + cols;
             if (quarter * 32 < D) {
+                float* dq_rows = dq_head + (size_t)row0 * D;
+                const int nr = p.Nq - row0;   // rows of this block inside the head
+                if (nr >= 32) {
 #pragma unroll
-                for (int e = 0; e < T::kQRows; ++e)
-                    if (row0 + e < p.Nq)
-                        red_add_f32(dq_head + (size_t)(row0 + e) * D, __uint_as_float(v[e]));
+                    for (int e = 0; e < 32; ++e) red_add_f32(dq_rows + e * D, __uint_as_float(v[e]));
+                } else {
+#pragma unroll
+                    for (int e = 0; e < 32; ++e)
+                        if (e < nr) red_add_f32(dq_rows + e * D, __uint_as_float(v[e]));
+                }
             }
         }
-    } else {
+    } else if (warp < 8) {
         // --------------------- P^T and dS^T (warps 0-7: key row, 32-query half) --
         const int quarter = warp & 3;
         const int half = warp >> 2;
@@ -461,7 +484,7 @@ __global__ void __launch_bounds__(448, 1)
     tc_fence_before_sync();
     __syncthreads();
     tc_fence_after_sync();
-    if (warp == 13) {
+    if (warp == 17) {
         tmem_dealloc(tbase, T::kTmemCols);
     }
 }

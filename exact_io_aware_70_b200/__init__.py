@@ -14,6 +14,8 @@ Entry points (same names as the C ABI):
   attn_lse_merge(o_part, lse_part, o, lse)
   attn_decode_splitkv(q, k, v, o, lse, scale, num_splits, workspace)
   attn_decode_workspace_bytes(B, H, d, num_splits)
+  attn_decode_paged(q, k_cache, v_cache, block_table, seq_lens, o, lse, scale, num_splits,
+                    workspace)                        paged-KV split-KV decode
   attn_status(stream) / attn_strerror(code)
 Tensor arguments are torch tensors on the current CUDA device (bf16 for
 q/k/v/o, fp32 for lse and partials, contiguous); ``stream`` defaults to torch's

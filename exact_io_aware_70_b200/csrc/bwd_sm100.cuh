@@ -197,8 +197,19 @@ __global__ void __launch_bounds__(640, 1)
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-    const int j = blockIdx.x;          // key block
-    const int bh = blockIdx.y;
+    // Launch order (x fastest, then y) -> (key block, head): heads in groups of
+    // kHeadGroup, and within a group the key blocks in order, each for every head
+    // of the group. Under the causal mask the early key blocks are the heavy ones,
+    // so the CTAs left to run at the end are light, while the CTAs resident at
+    // one time still share a few heads' Q and dO in L2.
+    constexpr int kHeadGroup = 4;
+    const int nkb = gridDim.x;
+    const int lin = blockIdx.y * nkb + blockIdx.x;
+    const int grp = lin / (kHeadGroup * nkb);
+    const int heads_in_grp = min(kHeadGroup, p.BH - grp * kHeadGroup);
+    const int rem = lin - grp * kHeadGroup * nkb;
+    const int j = rem / heads_in_grp;                       // key block
+    const int bh = grp * kHeadGroup + rem % heads_in_grp;
     const int i0 = bwd_first_qblock<CAUSAL>(j, p);
     const int nqb = (p.Nq + T::kQRows - 1) / T::kQRows;
     const int nsteps = nqb > i0 ? nqb - i0 : 0;

@@ -53,3 +53,15 @@ def test_reference_arm_prints_the_contract_line():
     assert cb["kind"] == "oracle" and cb["cores"] >= 1 and cb["sample"] and cb["value"] == line["value"]
     assert line["e2e"] == {"value": line["value"], "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
                            "d2h_bytes_per_step": 0}
+
+
+def test_l2_flush_plan():
+    """Inputs that fit in L2 are flushed before every timed step; larger ones are not."""
+    import bench
+    l2 = 126 << 20
+    on, note = bench.l2_flush_plan(50_700_000, l2, False)       # gpt2_1k forward
+    assert on and "fit in L2" in note and "flush" in note
+    on, note = bench.l2_flush_plan(192 << 20, l2, False)        # prefill_8k forward
+    assert not on and "larger than L2" in note
+    on, note = bench.l2_flush_plan(1 << 10, l2, True)           # reduced batch for profiling
+    assert not on and note == "reduced batch for profiling"

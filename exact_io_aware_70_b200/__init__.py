@@ -33,7 +33,7 @@ LIB_PATH = os.environ.get("EXACT_ATTN_LIB") or os.path.join(_HERE, "libexact_att
 
 if not os.path.exists(LIB_PATH):
     raise ImportError(
-        f"{LIB_PATH} is missing: build it with `python -m exact_io_aware_70_b200.build` "
+        f"{LIB_PATH} is missing: build it with `python exact_io_aware_70_b200/build.py` "
         "(this package has no CPU or fallback path)")
 
 lib = ctypes.CDLL(LIB_PATH)

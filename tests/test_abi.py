@@ -15,7 +15,12 @@ HEADER = os.path.join(ROOT, "include", "exact_attn.h")
 
 @pytest.fixture(scope="module")
 def ea():
-    from exact_io_aware_70_b200 import build
+    # the build script is loaded by path: importing the package first would
+    # refuse to load without the library this builds
+    spec = importlib.util.spec_from_file_location(
+        "exact_attn_cuda_build", os.path.join(ROOT, "exact_io_aware_70_b200", "build.py"))
+    build = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(build)
     build.build()
     import exact_io_aware_70_b200 as m
     return m

@@ -72,6 +72,8 @@ def _parity(B, H, Nq, Nkv, d, causal, seed):
     (2, 3, 640, 640, 64, False),
     (1, 2, 2048, 2048, 128, False),   # long non-causal: 32 query steps per key block
     (1, 1, 1500, 4000, 64, True),     # Nq < Nkv at length
+    (1, 5, 200, 200, 128, True),      # 5 heads: a launch-order group of 4 and one of 1
+    (1, 3, 333, 777, 64, False),      # 3 heads (one partial group), 7 key blocks
 ])
 def test_bwd_matches_oracle(B, H, Nq, Nkv, d, causal):
     _parity(B, H, Nq, Nkv, d, causal, seed=Nq * 7 + Nkv + d + int(causal))

@@ -28,6 +28,8 @@ SWEEP = [
     (1, 1, 2048, 2048, 128, False), # long non-causal rows: many ring wraps
     (1, 2, 1536, 4096, 64, True),   # Nq < Nkv at length
     (2, 1, 3000, 1000, 128, True),  # Nq > Nkv at length: 2000 rows per head see no key
+    (8, 64, 100, 100, 128, False),  # 512 units: several persistent rounds, a partial last one
+    (4, 100, 257, 257, 64, True),   # 800 units of two sizes over 5.4 rounds
 ]
 
 

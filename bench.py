@@ -107,9 +107,16 @@ def merge_bytes(w):
 
 # ---------------------------------------------------------------- helpers --
 def dist_env():
-    from exact_io_aware_70_b200.replicas import rank_info
-    r = rank_info()
-    return r.world_size, r.rank, r.local_rank
+    """(world size, rank, local rank) as torch.distributed.run sets them.
+
+    Parsed here rather than through the library's package, so that the
+    reference arm (the CPU oracle) never loads the CUDA library."""
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", str(rank)))
+    if ws < 1 or not 0 <= rank < ws:
+        raise ValueError(f"bad rank {rank} for world size {ws}")
+    return ws, rank, local
 
 
 def l2_flush_plan(resident_bytes, l2_bytes, reduced_batch):

@@ -1,8 +1,11 @@
 // attn_api.cu -- the C ABI declared in include/exact_attn.h.
 //
 // Argument checking, TMA tensor-map encoding and kernel launches. This is the
-// only translation unit of the library: the kernels live in the .cuh files it
-// includes, so the device status word below has a single definition.
+// only translation unit of the library that includes the kernels (they live
+// in the .cuh files below) and defines the device status word, so that word
+// has a single definition. The library's other translation unit,
+// attn_noalloc.cu, holds the allocation-free decode's scratch array and calls
+// only the extern "C" entry points defined here.
 #include <cuda.h>
 #include <cuda_runtime.h>
 

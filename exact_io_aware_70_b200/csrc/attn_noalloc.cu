@@ -10,6 +10,9 @@
 // array that belongs to this library's module, so the caller passes only the
 // inputs and outputs.
 //
+// This translation unit holds only that array and the entry point; it calls
+// the library's other extern "C" entry points and includes no kernel.
+//
 // Properties a user must know:
 //   * The array is kDecodeScratchBytes (32 MiB) on every GPU that loads this
 //     library, held until the process exits. Calls whose partials would not
@@ -19,12 +22,17 @@
 //     every entry the merge kernel reads. Calls that overlap on the GPU (for
 //     example on two streams at once) race on the array and give wrong
 //     results; serialise them.
-//   * The first call on each device looks up the array's device address with
-//     cudaGetSymbolAddress (host code cannot use the symbol itself: on the host
-//     it is only a stand-in, not a device address). Make that first call before
-//     any stream capture begins.
+//   * The first call in each CUDA context looks up the array's device address
+//     with cudaGetSymbolAddress (host code cannot use the symbol itself: on the
+//     host it is only a stand-in, not a device address). Make that first call
+//     before any stream capture begins. The address is cached per device
+//     together with the context's unique id, so a context that was torn down
+//     and created again (cudaDeviceReset, for instance) gets a fresh lookup
+//     instead of a stale address.
+#include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <cmath>
 #include <cstdint>
 #include <mutex>
 
@@ -37,22 +45,66 @@ constexpr int kMaxDevices = 64;
 
 static __device__ __align__(256) unsigned char g_decode_scratch[kDecodeScratchBytes];
 
-void* g_scratch_ptr[kMaxDevices] = {};
+struct ScratchSlot {
+    unsigned long long ctx_id = 0;   // id of the context the address belongs to
+    void* ptr = nullptr;
+};
+ScratchSlot g_scratch[kMaxDevices];
 std::mutex g_scratch_mu;
 
-// Device address of this device's scratch array (set up once per device, with
-// that device current). Returns nullptr if the lookup failed.
-void* scratch_for_current_device() {
+typedef CUresult (*CtxGetCurrentFn)(CUcontext*);
+typedef CUresult (*CtxGetIdFn)(CUcontext, unsigned long long*);
+
+template <class Fn>
+Fn driver_fn(const char* name) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion(name, &p, 12000, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+        return nullptr;
+    return reinterpret_cast<Fn>(p);
+}
+
+// Unique id of the calling thread's current context (0 if none is current).
+bool current_ctx_id(unsigned long long* id) {
+    static CtxGetCurrentFn get_current = nullptr;
+    static CtxGetIdFn get_id = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        get_current = driver_fn<CtxGetCurrentFn>("cuCtxGetCurrent");
+        get_id = driver_fn<CtxGetIdFn>("cuCtxGetId");
+    });
+    if (!get_current || !get_id) return false;
+    CUcontext ctx = nullptr;
+    if (get_current(&ctx) != CUDA_SUCCESS) return false;
+    if (ctx == nullptr) {
+        *id = 0;
+        return true;
+    }
+    return get_id(ctx, id) == CUDA_SUCCESS;
+}
+
+// Device address of the scratch array in the current context, with the
+// device current. Returns nullptr if the lookup failed.
+void* scratch_for_current_context() {
     int dev = -1;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
     std::lock_guard<std::mutex> lk(g_scratch_mu);
-    if (g_scratch_ptr[dev] == nullptr) {
-        void* ptr = nullptr;
-        if (cudaGetSymbolAddress(&ptr, g_decode_scratch) != cudaSuccess) return nullptr;
-        g_scratch_ptr[dev] = ptr;
-    }
-    return g_scratch_ptr[dev];
+    unsigned long long id = 0;
+    if (!current_ctx_id(&id)) return nullptr;
+    ScratchSlot& s = g_scratch[dev];
+    if (id != 0 && s.ptr != nullptr && s.ctx_id == id) return s.ptr;
+    // First use in this context (or no context yet: the lookup below makes the
+    // runtime create the device's primary context and make it current).
+    void* ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, g_decode_scratch) != cudaSuccess) return nullptr;
+    if (!current_ctx_id(&id) || id == 0) return nullptr;
+    s.ctx_id = id;
+    s.ptr = ptr;
+    return ptr;
 }
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
 }  // namespace
 
@@ -60,13 +112,23 @@ extern "C" attn_status_t attn_decode_splitkv_noalloc(const void* q, const void* 
                                                      void* o, float* lse, int B, int H, int Nkv,
                                                      int d, float scale, int num_splits,
                                                      void* stream) {
-    // Same arguments as attn_decode_splitkv, minus the workspace.
-    if (B < 1 || H < 1 || num_splits < 1) return ATTN_ERR_INVALID_ARG;
+    // Same arguments and checks as attn_decode_splitkv, minus the workspace.
+    // Every argument is checked here, before anything is enqueued, so that no
+    // partial kernel is launched into the shared array for a call that the
+    // merge step would then refuse.
+    if (!q || !k || !v || !o || !lse) return ATTN_ERR_INVALID_ARG;
+    if (!(scale > 0.f) || !std::isfinite(scale)) return ATTN_ERR_INVALID_ARG;
+    if (B < 1 || H < 1 || Nkv < 1 || Nkv > (1 << 30)) return ATTN_ERR_INVALID_ARG;
+    if ((long long)B * H > 65535) return ATTN_ERR_INVALID_ARG;   // grid.y of both kernels
+    if (num_splits < 1 || num_splits > 65535) return ATTN_ERR_INVALID_ARG;
     if (d != 64 && d != 128) return ATTN_ERR_UNSUPPORTED;
+    if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 2) ||
+        !aligned(lse, 4))
+        return ATTN_ERR_ALIGNMENT;
     const size_t need = attn_decode_workspace_bytes(B, H, d, num_splits);
     if (need == 0) return ATTN_ERR_INVALID_ARG;
     if (need > kDecodeScratchBytes) return ATTN_ERR_SCRATCH_LIMIT;
-    void* scratch = scratch_for_current_device();
+    void* scratch = scratch_for_current_context();
     if (scratch == nullptr) return ATTN_ERR_CUDA;
     // Partials layout as in attn_decode_splitkv: O_c first, then lse_c, each
     // rounded up to 256 bytes.

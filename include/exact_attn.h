@@ -214,13 +214,20 @@ attn_status_t attn_decode_paged(const void *q, const void *k_cache, const void *
  * over a device buffer, e.g. code inside an allocator's callbacks or a plugin
  * whose host framework owns all device memory.
  *
- *   Returns ATTN_ERR_SCRATCH_LIMIT, without launching, when the partials
- *   (attn_decode_workspace_bytes(B, H, d, num_splits) bytes) exceed 32 MiB.
+ *   Every argument is checked before anything is launched, with the codes
+ *   attn_decode_splitkv returns (null q, k, v, o or lse, B * H > 65535 or
+ *   num_splits > 65535: ATTN_ERR_INVALID_ARG; misaligned pointers:
+ *   ATTN_ERR_ALIGNMENT). Returns ATTN_ERR_SCRATCH_LIMIT, also without
+ *   launching, when the partials (attn_decode_workspace_bytes(B, H, d,
+ *   num_splits) bytes) exceed 32 MiB.
  *   All calls on a device share the array: calls that overlap on the GPU race
  *   and must be serialised by the caller. The array keeps the last call's
  *   contents; none of it needs to start at zero.
- *   The first call on each device looks up the array's device address
+ *   The first call in each CUDA context looks up the array's device address
  *   (cudaGetSymbolAddress); make that first call before any stream capture.
+ *   The address is cached with the context's unique id, so a context that is
+ *   destroyed and created again (e.g. after cudaDeviceReset) is looked up
+ *   afresh.
  */
 attn_status_t attn_decode_splitkv_noalloc(const void *q, const void *k, const void *v, void *o,
                                           float *lse, int B, int H, int Nkv, int d, float scale,

@@ -96,6 +96,38 @@ def test_decode_and_merge_reject_bad_arguments(ea):
     assert L.attn_decode_splitkv(p, p, p, p, p, 2, 3, 64, 96, 0.1, 8, p, need, None) == 2
 
 
+def test_noalloc_decode_rejects_bad_arguments_before_launching(ea):
+    """Every argument error of the allocation-free decode is returned before its
+    partial kernel is enqueued into the shared scratch array (the pointers are
+    never dereferenced; no GPU is needed)."""
+    f = ea.lib.attn_decode_splitkv_noalloc
+    f.restype = ctypes.c_int
+    f.argtypes = [ctypes.c_void_p] * 5 + [ctypes.c_int] * 4 + [ctypes.c_float, ctypes.c_int,
+                                                               ctypes.c_void_p]
+    p = 0x10000
+
+    def call(**kw):
+        a = dict(dict(q=p, k=p, v=p, o=p, lse=p, B=2, H=3, Nkv=64, d=128, scale=0.088, S=8),
+                 **kw)
+        return f(a["q"], a["k"], a["v"], a["o"], a["lse"], a["B"], a["H"], a["Nkv"], a["d"],
+                 a["scale"], a["S"], None)
+
+    assert call(o=None) == ea.ATTN_ERR_INVALID_ARG
+    assert call(lse=None) == ea.ATTN_ERR_INVALID_ARG
+    assert call(q=None) == ea.ATTN_ERR_INVALID_ARG
+    assert call(Nkv=0) == ea.ATTN_ERR_INVALID_ARG
+    assert call(S=0) == ea.ATTN_ERR_INVALID_ARG
+    assert call(S=65536) == ea.ATTN_ERR_INVALID_ARG
+    assert call(B=256, H=256) == ea.ATTN_ERR_INVALID_ARG      # B*H beyond the grid's y limit
+    assert call(scale=float("inf")) == ea.ATTN_ERR_INVALID_ARG
+    assert call(d=96) == ea.ATTN_ERR_UNSUPPORTED
+    assert call(o=p + 1) == ea.ATTN_ERR_ALIGNMENT
+    assert call(lse=p + 2) == ea.ATTN_ERR_ALIGNMENT
+    assert call(k=p + 8) == ea.ATTN_ERR_ALIGNMENT
+    # partials of 16 x 128 heads x 64 chunks (67.6 MB) exceed the fixed array
+    assert call(B=16, H=128, Nkv=32768, S=64) == ea.ATTN_ERR_SCRATCH_LIMIT
+
+
 def test_bwd_rejects_bad_arguments_without_launching(ea):
     L = ea.lib
     p = 0x10000

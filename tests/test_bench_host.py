@@ -65,3 +65,24 @@ def test_l2_flush_plan():
     assert not on and "larger than L2" in note
     on, note = bench.l2_flush_plan(1 << 10, l2, True)           # reduced batch for profiling
     assert not on and note == "reduced batch for profiling"
+
+
+def test_reference_arm_never_loads_the_cuda_library():
+    """The oracle arm shares no process image with the product: after a full
+    reference run neither the package nor its shared library is loaded."""
+    code = (
+        "import runpy, sys\n"
+        f"sys.argv = ['bench.py', '--impl', 'reference', '--steps', '1', '--warmup', '0']\n"
+        "try:\n"
+        f"    runpy.run_path({os.path.join(ROOT, 'bench.py')!r}, run_name='__main__')\n"
+        "except SystemExit as e:\n"
+        "    assert not e.code, e.code\n"
+        "maps = open('/proc/self/maps').read()\n"
+        "assert 'libexact_attn_b200' not in maps, 'CUDA library mapped'\n"
+        "assert not any(m.startswith('exact_io_aware_70_b200') for m in sys.modules)\n"
+        "assert 'liboracle' in maps\n"
+        "print('CLEAN')\n")
+    out = subprocess.run([sys.executable, "-c", code], capture_output=True, text=True,
+                         timeout=600, cwd=ROOT)
+    assert out.returncode == 0, out.stderr[-2000:]
+    assert "CLEAN" in out.stdout

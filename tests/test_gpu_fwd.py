@@ -78,17 +78,42 @@ def test_gpt2_1k_workload_full():
                              guard=0)
 
 
+def unit_rows(N, rng):
+    """Rows to check in one head of a long launch: the first and last row, one
+    random row inside every 256-row work unit (so every unit of every head is
+    looked at), and the two rows on either side of one random unit boundary and
+    of one random 128-row tile boundary."""
+    rows = {0, N - 1}
+    for u in range(0, N, 256):
+        rows.add(int(min(N - 1, u + rng.integers(0, 256))))
+    u = int(rng.integers(1, max(2, N // 256))) * 256
+    t = int(rng.integers(0, max(1, N // 256))) * 256 + 128
+    rows |= {u - 1, u, t - 1, t}
+    return sorted(r for r in rows if 0 <= r < N)
+
+
 @pytest.mark.parametrize("name", ["prefill_8k", "prefill_16k"])
-def test_long_prefill_sampled(name):
+def test_long_prefill_every_head(name):
+    """The full-size launch in the configuration bench.py times, checked in
+    every (batch, head): a head-, unit- or round-indexing mistake anywhere in
+    the persistent schedule shows up as a wrong row somewhere."""
+    import oracle
+    from seeded_inputs import bf16_bits
+    from tests.parity import compare
     w = WORKLOADS[name]
     q, k, v = make_workload(w, device="cuda")
     o, lse = gpu_util.run_fwd(q, k, v, w.causal, w.scale)
+    assert torch.isfinite(o.float()).all() and torch.isfinite(lse).all()
+    orc = oracle.get()
     rng = np.random.default_rng(w.seed)
-    heads = [(0, 0), (w.B - 1, w.H - 1), (w.B // 2, w.H // 2)]
-    gpu_util.fwd_sampled_parity(q, k, v, o, lse, w.causal, w.scale, heads, rng)
-    # properties at every row: finite O, LSE at least the log of the visible count's lower bound
-    assert torch.isfinite(o.float()).all()
-    assert torch.isfinite(lse).all()
+    qc, kc, vc, oc, lc = (t.cpu() for t in (q, k, v, o, lse))
+    for b in range(w.B):
+        for h in range(w.H):
+            rows = unit_rows(w.Nq, rng)
+            o_ref, l_ref = orc.attn_rows_bf16(bf16_bits(qc[b, h]), bf16_bits(kc[b, h]),
+                                              bf16_bits(vc[b, h]), rows, w.causal, w.scale)
+            compare(oc[b, h, rows].float().numpy(), lc[b, h, rows].numpy(), o_ref, l_ref,
+                    f"{name} head ({b},{h})")
 
 
 def test_deterministic():

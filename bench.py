@@ -119,6 +119,16 @@ def dist_env():
     return ws, rank, local
 
 
+def rank_slice(w, rank):
+    """This rank's slice of a workload that grows with the number of GPUs: the
+    same shapes, drawn from the rank's own seed (its own batch entries for a
+    prefill, its own shard of the keys for a decode)."""
+    import dataclasses
+
+    from exact_io_aware_70_b200.sharding import shard_seed
+    return dataclasses.replace(w, seed=shard_seed(w.seed, rank))
+
+
 def l2_flush_plan(resident_bytes, l2_bytes, reduced_batch):
     """(flush?, note) for a timed loop. Inputs that fit in L2 would be served from
     it when run back to back, so such workloads are timed cold: a buffer of twice
@@ -296,8 +306,9 @@ def recorded_traffic():
 
 
 # ------------------------------------------------------------ CPU oracle --
-def oracle_prefill_sample(budget_s, max_rows=None, max_heads=4):
-    """Time the oracle on evenly spaced query rows of the prefill workload's heads.
+def oracle_prefill_sample(budget_s, max_rows=None, max_heads=4, w=None):
+    """Time the oracle on evenly spaced query rows of a prefill workload's heads
+    (prefill_8k unless `w` names another).
 
     The row count grows until one head's sample takes a quarter of the budget
     (or covers every row); whole heads are then repeated while the budget lasts.
@@ -306,7 +317,7 @@ def oracle_prefill_sample(budget_s, max_rows=None, max_heads=4):
 
     import oracle
     from seeded_inputs import bf16_bits, make_qkv
-    w = PREFILL
+    w = PREFILL if w is None else w
     orc = oracle.get()
     q, k, v = make_qkv(1, max_heads, w.Nq, w.Nkv, w.d, w.seed)   # CPU generator
     hb = [(bf16_bits(q[0, h]), bf16_bits(k[0, h]), bf16_bits(v[0, h])) for h in range(max_heads)]
@@ -325,7 +336,8 @@ def oracle_prefill_sample(budget_s, max_rows=None, max_heads=4):
         orc.attn_rows_bf16(*hb[heads], rows, w.causal, w.scale)
         dt += time.perf_counter() - t0
         heads += 1
-    flops = heads * sum(4.0 * w.d * min(w.Nkv, int(r) + 1 + (w.Nkv - w.Nq)) for r in rows)
+    flops = heads * sum(4.0 * w.d * (min(w.Nkv, max(0, int(r) + 1 + (w.Nkv - w.Nq)))
+                                     if w.causal else w.Nkv) for r in rows)
     return {"flops": flops, "seconds": dt, "rows": int(nrows), "heads": heads,
             "cores": orc.num_threads()}
 
@@ -361,6 +373,8 @@ def cpu_baseline(budget_s=8.0):
                    f"decode: {dc['heads']} (b,h) rows of decode_32k "
                    f"({dc['bytes'] / 1e9:.2f} GB of K/V in {dc['seconds']:.2f} s)"),
         "decode": {"value": dc["bytes"] / dc["seconds"] / 1e9, "unit": "GB/s"},
+        "decode_sample": (f"fp64 oracle, {dc['heads']} (b,h) rows of decode_32k "
+                          f"({dc['bytes'] / 1e9:.2f} GB of K/V in {dc['seconds']:.2f} s)"),
     }
 
 
@@ -529,7 +543,7 @@ def run_fp8(args):
     import torch.distributed as dist
 
     import exact_io_aware_70_b200 as ea
-    from exact_io_aware_70_b200.replicas import max_over_ranks, replica_workload
+    from exact_io_aware_70_b200.sharding import max_over_ranks
     from seeded_inputs import make_qkv_fp8
 
     ws, rank, local = dist_env()
@@ -543,7 +557,7 @@ def run_fp8(args):
     sp = stream.cuda_stream
     L = ea.lib
     w = _maybe_batch(WORKLOADS[args.workload[:-len("_fp8")]], args.batch)
-    wr = replica_workload(w, rank)
+    wr = rank_slice(w, rank)
     ins = make_qkv_fp8(w.B, w.H, w.Nq, w.Nkv, w.d, wr.seed, device="cuda")
     o = torch.empty((w.B, w.H, w.Nq, w.d), dtype=torch.bfloat16, device=dev)
     lse = torch.empty((w.B, w.H, w.Nq), dtype=torch.float32, device=dev)
@@ -624,7 +638,8 @@ def run_fp8(args):
         "vs_baseline": None, "dtype": "e4m3", "data": "synthetic",
         "config": {"workload": args.workload, "B": w.B, "H": w.H, "N": w.Nq, "d": w.d,
                    "causal": w.causal, "flop_per_step": prefill_flops(w), "l2": flush.note,
-                   "parallelism": f"replicas x{ws}" if ws > 1 else "1 GPU"},
+                   "parallelism": (f"batch partitioned: one {w.B}-entry slice per GPU x{ws}"
+                                   if ws > 1 else "1 GPU")},
         "roofline": roof,
         "peaks": dict(pk, note="of measured" if pk["source"] == "measured" else "of fallback"),
         "clocks": clk.summary(max_mhz_default=1965.0),
@@ -651,7 +666,7 @@ def run_bwd(args):
     import torch.distributed as dist
 
     import exact_io_aware_70_b200 as ea
-    from exact_io_aware_70_b200.replicas import max_over_ranks, replica_workload
+    from exact_io_aware_70_b200.sharding import max_over_ranks
     from seeded_inputs import make_dout
 
     ws, rank, local = dist_env()
@@ -665,7 +680,7 @@ def run_bwd(args):
     sp = stream.cuda_stream
     L = ea.lib
     w = _maybe_batch(WORKLOADS[args.workload[:-len("_bwd")]], args.batch)
-    wr = replica_workload(w, rank)
+    wr = rank_slice(w, rank)
     q, k, v = make_workload(wr, device="cuda")
     do = make_dout(w.B, w.H, w.Nq, w.d, wr.seed, device="cuda")
     o = torch.empty_like(q)
@@ -749,7 +764,8 @@ def run_bwd(args):
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": {"workload": args.workload, "B": w.B, "H": w.H, "N": w.Nq, "d": w.d,
                    "causal": w.causal, "flop_per_step": bwd_flops(w), "l2": flush.note,
-                   "parallelism": f"replicas x{ws}" if ws > 1 else "1 GPU"},
+                   "parallelism": (f"batch partitioned: one {w.B}-entry slice per GPU x{ws}"
+                                   if ws > 1 else "1 GPU")},
         "roofline": roof,
         "peaks": dict(pk, note="of measured" if pk["source"] == "measured" else "of fallback"),
         "clocks": clk.summary(max_mhz_default=1965.0),
@@ -775,13 +791,84 @@ def _maybe_batch(w, batch):
     return dataclasses.replace(w, B=batch) if batch else w
 
 
-def run_ours(args):
-    import dataclasses
+def _peaks_note(pk):
+    return "of measured" if pk["source"] == "measured" else "of fallback"
 
+
+def prefill_roofline(w, ms, pk, traffic=None):
+    a = prefill_flops(w) / (ms * 1e-3) / 1e12
+    return {"bound": "tensor", "achieved": a, "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
+            "frac": a / pk["bf16_tflops"], "frac_of_sustained": a / pk["bf16_tflops_sustained"],
+            "traffic": traffic, "algorithmic_bytes": prefill_bytes(w),
+            "algorithmic_flops": prefill_flops(w), "ms": ms, "note": _peaks_note(pk)}
+
+
+def prefill_cpu_baseline(w, budget_s):
+    cb = oracle_prefill_sample(budget_s, max_heads=min(4, w.H), w=w)
+    return {"value": cb["flops"] / cb["seconds"] / 1e12, "unit": "TFLOP/s", "cores": cb["cores"],
+            "kind": "oracle",
+            "sample": (f"fp64 oracle, {cb['rows']} evenly spaced query rows of each of "
+                       f"{cb['heads']} heads of {w.name} ({cb['flops'] / 1e9:.2f} GFLOP in "
+                       f"{cb['seconds']:.2f} s)")}
+
+
+def time_prefill_workload(ea, w, K, warmup, dev, stream, local, cpu_budget):
+    """One more prefill workload of the default line, timed on its own after
+    the step: K calls of attn_fwd (cold L2 where the inputs fit in it, with the
+    hot figure alongside), its roofline and the oracle on a bounded sample."""
+    import torch
+    q, k, v = make_workload(w, device="cuda")
+    o = torch.empty_like(q)
+    lse = torch.empty((w.B, w.H, w.Nq), dtype=torch.float32, device=dev)
+    sp = stream.cuda_stream
+    args_c = (q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(), w.B, w.H,
+              w.Nq, w.Nkv, w.d, int(w.causal), w.scale, sp)
+
+    def step():
+        rc = ea.lib.attn_fwd(*args_c)
+        if rc != 0:
+            raise RuntimeError(f"attn_fwd ({w.name}): {ea.attn_strerror(rc)}")
+
+    flush = L2Flusher([q, k, v, o, lse], dev, False)
+    for _ in range(warmup):
+        step()
+    if ea.attn_status() != 0:
+        raise RuntimeError(f"device status reported an error during {w.name} warm-up")
+    _, call_ms, clk, hot_ms = timed_calls(step, K, flush, stream, 1, local)
+    if ea.attn_status() != 0:
+        raise RuntimeError(f"device status reported an error timing {w.name}")
+    pk = peaks()
+    out = {"config": {"B": w.B, "H": w.H, "N": w.Nq, "d": w.d, "causal": w.causal,
+                      "seed": w.seed, "l2": flush.note},
+           "ms": call_ms, "value": prefill_flops(w) / (call_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+           "roofline": dict(prefill_roofline(w, call_ms, pk), kernel="attn_fwd_sm100"),
+           "clocks": clk.summary(max_mhz_default=1965.0), "gpu_launches": K}
+    if hot_ms is not None:
+        out["hot"] = {"ms": hot_ms, "value": prefill_flops(w) / (hot_ms * 1e-3) / 1e12,
+                      "unit": "TFLOP/s", "frac": prefill_flops(w) / (hot_ms * 1e-3) / 1e12
+                      / pk["bf16_tflops"], "note": "back to back, L2 not flushed"}
+    if cpu_budget > 0:
+        out["cpu_baseline"] = prefill_cpu_baseline(w, cpu_budget)
+    del q, k, v, o, lse
+    torch.cuda.empty_cache()
+    return out
+
+
+def run_ours(args):
+    """The default line: one step = prefill_8k forward + decode_32k split-KV
+    decode (partials + merge), plus, in the same run at one GPU, the other
+    workloads (tiny, gpt2_1k, prefill_16k) timed on their own.
+
+    With N GPUs (torchrun) the job grows with N (weak scaling): the prefill
+    batch has N entries, one per GPU (its heads partitioned over the ranks by
+    batch entry); the decode sequence has N x 32768 keys, one 32768-key shard
+    per GPU, whose partials are all-gathered (NCCL) and merged on every GPU
+    with attn_lse_merge_gathered."""
     import torch
     import torch.distributed as dist
 
     import exact_io_aware_70_b200 as ea
+    from exact_io_aware_70_b200.sharding import max_over_ranks
 
     ws, rank, local = dist_env()
     torch.cuda.set_device(local)
@@ -794,6 +881,7 @@ def run_ours(args):
     sp = stream.cuda_stream
     L = ea.lib
 
+    import dataclasses
     paged = args.workload == "decode_32k_paged"
     if args.workload == "step":
         pw, dw = PREFILL, DECODE
@@ -809,11 +897,10 @@ def run_ours(args):
     pw = _maybe_batch(pw, args.batch) if pw else None
     dw = _maybe_batch(dw, args.batch) if dw else None
 
-    # ---- inputs resident in HBM (seed offset per rank: each rank its own batch)
-    kernels = []
-    from exact_io_aware_70_b200.replicas import max_over_ranks, replica_workload
+    # ---- inputs resident in HBM; each rank draws its own slice of the job
+    kernels = []        # (name, launch, is_ours)
     if pw:
-        pw_r = replica_workload(pw, rank)
+        pw_r = rank_slice(pw, rank)
         q, k, v = make_workload(pw_r, device="cuda")
         o = torch.empty_like(q)
         lse = torch.empty((pw.B, pw.H, pw.Nq), dtype=torch.float32, device=dev)
@@ -822,52 +909,62 @@ def run_ours(args):
             return L.attn_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
                               lse.data_ptr(), pw.B, pw.H, pw.Nq, pw.Nkv, pw.d, int(pw.causal),
                               pw.scale, sp)
-        kernels.append(("attn_fwd_sm100", launch_prefill))
-    if dw and paged:
-        from seeded_inputs import PAGED_DECODE as PD, make_paged_cache
-        dw_r = replica_workload(dw, rank)
-        dq, dk, dv, dtable, dlens = make_paged_cache(dw.B, dw.H, [dw.Nkv] * dw.B, dw.d,
-                                                     PD["page_size"], dw_r.seed, device="cuda")
+        kernels.append(("attn_fwd_sm100", launch_prefill, True))
+    if dw:
+        S = dw.num_splits
+        dw_r = rank_slice(dw, rank)
+        if paged:
+            from seeded_inputs import PAGED_DECODE as PD, make_paged_cache
+            dq, dk, dv, dtable, dlens = make_paged_cache(dw.B, dw.H, [dw.Nkv] * dw.B, dw.d,
+                                                         PD["page_size"], dw_r.seed, device="cuda")
+            if ws > 1:   # the query row is the same on every rank; the cache is the rank's shard
+                dq = make_paged_cache(dw.B, dw.H, [dw.Nkv] * dw.B, dw.d, PD["page_size"],
+                                      dw.seed, device="cuda")[0]
+        else:
+            _, dk, dv = make_workload(dw_r, device="cuda")
+            dq = make_workload(dw, device="cuda")[0] if ws > 1 else make_workload(dw_r, "cuda")[0]
         do = torch.empty_like(dq)
         dlse = torch.empty((dw.B, dw.H, 1), dtype=torch.float32, device=dev)
-        S = dw.num_splits
         work = torch.empty(ea.attn_decode_workspace_bytes(dw.B, dw.H, dw.d, S), dtype=torch.uint8,
                            device=dev)
         o_bytes = ((dw.B * dw.H * S * dw.d * 4 + 255) // 256) * 256
-        o_part = work.data_ptr()
-        lse_part = work.data_ptr() + o_bytes
-        npages, ps = dk.shape[0], PD["page_size"]
+        if ws > 1:
+            # this rank's partials, and the buffers the all-gather fills (rank r at [r])
+            po = torch.empty((dw.B, dw.H, S, dw.d), dtype=torch.float32, device=dev)
+            pl = torch.empty((dw.B, dw.H, S), dtype=torch.float32, device=dev)
+            og = torch.empty((ws, dw.B, dw.H, S, dw.d), dtype=torch.float32, device=dev)
+            lg = torch.empty((ws, dw.B, dw.H, S), dtype=torch.float32, device=dev)
+            o_part, lse_part = po.data_ptr(), pl.data_ptr()
+        else:
+            o_part, lse_part = work.data_ptr(), work.data_ptr() + o_bytes
+        if paged:
+            npages, ps = dk.shape[0], PD["page_size"]
 
-        def launch_partials():
-            return L.attn_decode_paged_partials(dq.data_ptr(), dk.data_ptr(), dv.data_ptr(),
-                                                dtable.data_ptr(), dlens.data_ptr(), o_part,
-                                                lse_part, dw.B, dw.H, dw.d, ps, dtable.shape[1],
-                                                npages, dw.scale, S, sp)
+            def launch_partials():
+                return L.attn_decode_paged_partials(dq.data_ptr(), dk.data_ptr(), dv.data_ptr(),
+                                                    dtable.data_ptr(), dlens.data_ptr(), o_part,
+                                                    lse_part, dw.B, dw.H, dw.d, ps,
+                                                    dtable.shape[1], npages, dw.scale, S, sp)
+        else:
+            def launch_partials():
+                return L.attn_decode_partials(dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), o_part,
+                                              lse_part, dw.B, dw.H, dw.Nkv, dw.d, dw.scale, S, sp)
+        kernels.append(("attn_decode_partials", launch_partials, True))
+        if ws > 1:
+            def launch_gather():
+                dist.all_gather_into_tensor(og, po)
+                dist.all_gather_into_tensor(lg, pl)
+                return 0
 
-        def launch_merge():
-            return L.attn_lse_merge(o_part, lse_part, do.data_ptr(), dlse.data_ptr(), dw.B, dw.H,
-                                    S, dw.d, sp)
-        kernels += [("attn_decode_partials", launch_partials), ("attn_lse_merge", launch_merge)]
-    elif dw:
-        dw_r = replica_workload(dw, rank)
-        dq, dk, dv = make_workload(dw_r, device="cuda")
-        do = torch.empty_like(dq)
-        dlse = torch.empty((dw.B, dw.H, 1), dtype=torch.float32, device=dev)
-        S = dw.num_splits
-        work = torch.empty(ea.attn_decode_workspace_bytes(dw.B, dw.H, dw.d, S), dtype=torch.uint8,
-                           device=dev)
-        o_bytes = ((dw.B * dw.H * S * dw.d * 4 + 255) // 256) * 256
-        o_part = work.data_ptr()
-        lse_part = work.data_ptr() + o_bytes
-
-        def launch_partials():
-            return L.attn_decode_partials(dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), o_part,
-                                          lse_part, dw.B, dw.H, dw.Nkv, dw.d, dw.scale, S, sp)
-
-        def launch_merge():
-            return L.attn_lse_merge(o_part, lse_part, do.data_ptr(), dlse.data_ptr(), dw.B, dw.H,
-                                    S, dw.d, sp)
-        kernels += [("attn_decode_partials", launch_partials), ("attn_lse_merge", launch_merge)]
+            def launch_merge():
+                return L.attn_lse_merge_gathered(og.data_ptr(), lg.data_ptr(), do.data_ptr(),
+                                                 dlse.data_ptr(), ws, dw.B, dw.H, S, dw.d, sp)
+            kernels.append(("nccl_all_gather", launch_gather, False))
+        else:
+            def launch_merge():
+                return L.attn_lse_merge(o_part, lse_part, do.data_ptr(), dlse.data_ptr(), dw.B,
+                                        dw.H, S, dw.d, sp)
+        kernels.append(("attn_lse_merge", launch_merge, True))
     torch.cuda.synchronize()
     resident = ([q, k, v, o, lse] if pw else []) + ([dq, dk, dv, do, dlse, work] if dw else [])
     if dw and paged:
@@ -875,7 +972,7 @@ def run_ours(args):
     flush = L2Flusher(resident, dev, bool(args.batch))
 
     def step(evs=None):
-        for i, (name, fn) in enumerate(kernels):
+        for i, (name, fn, _) in enumerate(kernels):
             if evs is not None:
                 evs[i].record(stream)
             rc = fn()
@@ -899,9 +996,9 @@ def run_ours(args):
             dist.barrier()
         torch.cuda.synchronize()
         t_start.record(stream)
-        for s in range(K):
+        for s_ in range(K):
             flush()
-            step(ev[s])
+            step(ev[s_])
         t_end.record(stream)
         torch.cuda.synchronize()
         if ws > 1:
@@ -909,23 +1006,23 @@ def run_ours(args):
     if ea.attn_status() != 0:
         raise RuntimeError("device status reported an error in the timed region")
     total_ms = t_start.elapsed_time(t_end)
-    per_kernel_ms = [statistics.mean(ev[s][i].elapsed_time(ev[s][i + 1]) for s in range(K))
+    per_kernel_ms = [statistics.mean(ev[s_][i].elapsed_time(ev[s_][i + 1]) for s_ in range(K))
                      for i in range(len(kernels))]
     hot_kernel_ms = []
     if flush.active:
         # the same kernels back to back, L2 not flushed
-        for s in range(K):
-            step(ev[s])
+        for s_ in range(K):
+            step(ev[s_])
         torch.cuda.synchronize()
         if ea.attn_status() != 0:
             raise RuntimeError("device status reported an error in the hot region")
-        hot_kernel_ms = [statistics.mean(ev[s][i].elapsed_time(ev[s][i + 1]) for s in range(K))
+        hot_kernel_ms = [statistics.mean(ev[s_][i].elapsed_time(ev[s_][i + 1]) for s_ in range(K))
                          for i in range(len(kernels))]
     vals = max_over_ranks([total_ms] + per_kernel_ms + hot_kernel_ms, device=dev)
     total_ms, per_kernel_ms = vals[0], vals[1:1 + len(kernels)]
     hot_kernel_ms = vals[1 + len(kernels):]
-    kms = dict(zip([n for n, _ in kernels], per_kernel_ms))
-    hot_kms = dict(zip([n for n, _ in kernels], hot_kernel_ms))
+    kms = dict(zip([n for n, _, _ in kernels], per_kernel_ms))
+    hot_kms = dict(zip([n for n, _, _ in kernels], hot_kernel_ms))
 
     # ---- e2e: the same work through the public API from pinned host buffers
     e2e = None
@@ -956,7 +1053,15 @@ def run_ours(args):
             dq.copy_(hdq, non_blocking=True)
             dk.copy_(hdk, non_blocking=True)
             dv.copy_(hdv, non_blocking=True)
-            if paged:
+            if ws > 1:
+                # this rank's shard through the public API, then the exchange and the merge
+                if paged:
+                    ea.attn_decode_paged_partials(dq, dk, dv, dtable, dlens, po, pl, dw.scale, S)
+                else:
+                    ea.attn_decode_partials(dq, dk, dv, po, pl, dw.scale, S)
+                launch_gather()
+                ea.attn_lse_merge_gathered(og, lg, do, dlse)
+            elif paged:
                 ea.attn_decode_paged(dq, dk, dv, dtable, dlens, do, dlse, dw.scale, S, work)
             else:
                 ea.attn_decode_splitkv(dq, dk, dv, do, dlse, dw.scale, S, work)
@@ -1006,49 +1111,60 @@ def run_ours(args):
     step_ms = sum(per_kernel_ms)
     roof = {}
     if pw:
-        t = kms["attn_fwd_sm100"]
-        a = prefill_flops(pw) / (t * 1e-3) / 1e12
-        roof["attn_fwd_sm100"] = {
-            "bound": "tensor", "achieved": a, "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
-            "frac": a / pk["bf16_tflops"], "frac_of_sustained": a / pk["bf16_tflops_sustained"],
-            "traffic": traffic.get("attn_fwd_sm100"), "algorithmic_bytes": prefill_bytes(pw),
-            "algorithmic_flops": prefill_flops(pw), "ms": t, "share": t / step_ms}
+        roof["attn_fwd_sm100"] = dict(prefill_roofline(pw, kms["attn_fwd_sm100"], pk,
+                                                       traffic.get("attn_fwd_sm100")),
+                                      share=kms["attn_fwd_sm100"] / step_ms)
     if dw:
+        mbytes = merge_bytes(dw) * ws
         for name, nbytes in (("attn_decode_partials", decode_partial_bytes(dw)),
-                             ("attn_lse_merge", merge_bytes(dw))):
+                             ("attn_lse_merge", mbytes)):
             t = kms[name]
             a = nbytes / (t * 1e-3) / 1e9
             roof[name] = {"bound": "hbm", "achieved": a, "peak": pk["hbm_gbs"], "unit": "GB/s",
                           "frac": a / pk["hbm_gbs"], "traffic": traffic.get(name),
-                          "algorithmic_bytes": nbytes, "ms": t, "share": t / step_ms}
+                          "algorithmic_bytes": nbytes, "ms": t, "share": t / step_ms,
+                          "note": _peaks_note(pk)}
     dominant = max(roof, key=lambda n: roof[n]["ms"])
     dom = dict(roof[dominant], kernel=dominant)
+    if ws > 1:
+        par = []
+        if pw:
+            par.append(f"prefill: heads partitioned, one {pw.B}x{pw.H}-head batch slice per GPU")
+        if dw:
+            par.append(f"decode: KV sequence split, one {dw.Nkv}-key shard per GPU, partials "
+                       "all-gathered (NCCL) and merged on every GPU")
+        parallelism = f"{ws} GPUs; " + "; ".join(par)
+    else:
+        parallelism = "1 GPU"
     cfg = {"workload": "prefill_8k + decode_32k" if args.workload == "step" else args.workload,
-           "l2": flush.note, "parallelism": f"replicas x{ws}" if ws > 1 else "1 GPU"}
+           "l2": flush.note, "parallelism": parallelism}
     line = {"metric": METRIC}
     if pw:
         pf = kms["attn_fwd_sm100"]
-        cfg["prefill"] = {"B": pw.B, "H": pw.H, "N": pw.Nq, "d": pw.d, "causal": pw.causal,
-                          "flop_per_step": prefill_flops(pw)}
+        cfg["prefill"] = {"B": pw.B * ws, "H": pw.H, "N": pw.Nq, "d": pw.d, "causal": pw.causal,
+                          "flop_per_step": ws * prefill_flops(pw)}
         line.update(value=ws * prefill_flops(pw) / (pf * 1e-3) / 1e12, unit="TFLOP/s")
         line["prefill"] = {"value": line["value"], "unit": "TFLOP/s", "ms": pf,
                            "frac_of_bf16_peak": roof["attn_fwd_sm100"]["frac"]}
     if dw:
-        dms = kms["attn_decode_partials"] + kms["attn_lse_merge"]
-        cfg["decode"] = {"B": dw.B, "H": dw.H, "Nkv": dw.Nkv, "d": dw.d, "splits": dw.num_splits,
-                         "kv_bytes_per_step": decode_kv_bytes(dw)}
+        dnames = ["attn_decode_partials", "attn_lse_merge"] + (["nccl_all_gather"] if ws > 1 else [])
+        dms = sum(kms[n] for n in dnames)
+        cfg["decode"] = {"B": dw.B, "H": dw.H, "Nkv": dw.Nkv * ws, "d": dw.d,
+                         "splits": dw.num_splits * ws, "kv_bytes_per_step": ws * decode_kv_bytes(dw)}
         dgbs = decode_kv_bytes(dw) / (dms * 1e-3) / 1e9
         line["decode"] = {"value": ws * dgbs, "unit": "GB/s", "ms": dms,
                           "frac_of_hbm_peak": dgbs / pk["hbm_gbs"]}
+        if ws > 1:
+            line["decode"]["all_gather_ms"] = kms["nccl_all_gather"]
         if not pw:
             line.update(value=ws * dgbs, unit="GB/s")
     line.update({
         "n_gpus": ws, "steps": K, "warmup": args.warmup, "ms_per_step": total_ms / K,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic", "config": cfg, "roofline": dom, "roofline_kernels": roof,
-        "peaks": dict(pk, note="of measured" if pk["source"] == "measured" else "of fallback"),
+        "peaks": dict(pk, note=_peaks_note(pk)),
         "clocks": clk.summary(max_mhz_default=1965.0),
-        "gpu_launches": len(kernels) * K, "e2e": e2e,
+        "gpu_launches": sum(1 for _, _, ours in kernels if ours) * K, "e2e": e2e,
     })
     if hot_kms:
         hot = {"ms": sum(hot_kms.values()), "note": "the same kernels back to back, L2 not flushed"}
@@ -1058,8 +1174,42 @@ def run_ours(args):
         else:
             hot.update(value=ws * decode_kv_bytes(dw) / (hot["ms"] * 1e-3) / 1e9, unit="GB/s")
         line["hot"] = hot
+    cb = None
     if ws == 1 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline(args.cpu_budget)
+        cb = cpu_baseline(args.cpu_budget)
+        line["cpu_baseline"] = cb
+    if ws == 1 and args.workload == "step" and not args.no_workloads:
+        # the five workloads, each with its own roofline and oracle baseline
+        wl = {}
+        for name in ("tiny", "gpt2_1k"):
+            wl[name] = time_prefill_workload(ea, WORKLOADS[name], K, args.warmup, dev, stream,
+                                             local, 0 if args.no_cpu_baseline else 2.0)
+        wl["prefill_8k"] = {
+            "config": {"B": pw.B, "H": pw.H, "N": pw.Nq, "d": pw.d, "causal": pw.causal,
+                       "seed": pw.seed, "l2": flush.note},
+            "ms": kms["attn_fwd_sm100"], "value": line["prefill"]["value"], "unit": "TFLOP/s",
+            "roofline": dict(roof["attn_fwd_sm100"], kernel="attn_fwd_sm100"),
+            "note": "timed inside the step (after the 8.6 GB decode of the previous step)"}
+        if cb:
+            wl["prefill_8k"]["cpu_baseline"] = {k_: cb[k_] for k_ in
+                                                ("value", "unit", "cores", "kind", "sample")}
+        wl["prefill_16k"] = time_prefill_workload(ea, WORKLOADS["prefill_16k"], max(3, K // 2),
+                                                  args.warmup, dev, stream, local,
+                                                  0 if args.no_cpu_baseline else 2.0)
+        wl["decode_32k"] = {
+            "config": {"B": dw.B, "H": dw.H, "Nkv": dw.Nkv, "d": dw.d, "splits": dw.num_splits,
+                       "seed": dw.seed, "l2": flush.note},
+            "ms": line["decode"]["ms"], "value": line["decode"]["value"], "unit": "GB/s",
+            "roofline": dict(roof["attn_decode_partials"], kernel="attn_decode_partials"),
+            "merge_roofline": dict(roof["attn_lse_merge"], kernel="attn_lse_merge"),
+            "frac_of_hbm_peak": line["decode"]["frac_of_hbm_peak"],
+            "note": "partials + merge, timed inside the step"}
+        if cb:
+            wl["decode_32k"]["cpu_baseline"] = dict(cb["decode"], cores=cb["cores"],
+                                                    kind="oracle", sample=cb["decode_sample"])
+        line["workloads"] = wl
+        line["gpu_launches"] += sum(w_["gpu_launches"] for w_ in wl.values()
+                                    if "gpu_launches" in w_)
     if ws == 1 and pw is PREFILL and not args.no_naive:
         line["naive_comparison"] = naive_comparison(dev, kms["attn_fwd_sm100"])
     print(json.dumps(line), flush=True)
@@ -1083,6 +1233,8 @@ def main():
                     help="override the batch size (small profiling captures only)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-workloads", action="store_true",
+                    help="default line only: skip timing tiny, gpt2_1k and prefill_16k")
     ap.add_argument("--no-naive", action="store_true",
                     help="skip the naive materialising attention comparison")
     ap.add_argument("--cpu-budget", type=float, default=8.0,

@@ -55,6 +55,8 @@ lib.attn_decode_partials.restype = _i
 lib.attn_decode_partials.argtypes = [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _f, _i, _vp]
 lib.attn_lse_merge.restype = _i
 lib.attn_lse_merge.argtypes = [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _vp]
+lib.attn_lse_merge_gathered.restype = _i
+lib.attn_lse_merge_gathered.argtypes = [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _vp]
 lib.attn_decode_workspace_bytes.restype = _sz
 lib.attn_decode_workspace_bytes.argtypes = [_i, _i, _i, _i]
 lib.attn_decode_splitkv.restype = _i
@@ -175,6 +177,21 @@ def attn_lse_merge(o_part, lse_part, o, lse, stream=None) -> None:
                               _tensor(lse_part, torch.float32, "lse_part"),
                               _tensor(o, torch.bfloat16, "o"), _tensor(lse, torch.float32, "lse"),
                               B, H, S, d, _stream(stream)), "attn_lse_merge")
+
+
+def attn_lse_merge_gathered(o_part, lse_part, o, lse, stream=None) -> None:
+    """Max-and-sum merge of partials gathered from R ranks' KV shards.
+    o_part [R,B,H,S,d], lse_part [R,B,H,S] fp32 -> o [B,H,1,d] bf16, lse [B,H,1] fp32."""
+    import torch
+    R, B, H, S, d = o_part.shape
+    if (tuple(lse_part.shape) != (R, B, H, S) or tuple(o.shape) != (B, H, 1, d)
+            or tuple(lse.shape) != (B, H, 1)):
+        raise ValueError("attn_lse_merge_gathered: inconsistent shapes")
+    _check(lib.attn_lse_merge_gathered(_tensor(o_part, torch.float32, "o_part"),
+                                       _tensor(lse_part, torch.float32, "lse_part"),
+                                       _tensor(o, torch.bfloat16, "o"),
+                                       _tensor(lse, torch.float32, "lse"),
+                                       R, B, H, S, d, _stream(stream)), "attn_lse_merge_gathered")
 
 
 def attn_decode_workspace_bytes(B: int, H: int, d: int, num_splits: int) -> int:

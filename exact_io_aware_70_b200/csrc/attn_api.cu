@@ -395,24 +395,54 @@ attn_status_t attn_decode_paged(const void* q, const void* k_cache, const void* 
     return attn_lse_merge(o_part, lse_part, o, lse, B, H, num_splits, d, stream);
 }
 
-attn_status_t attn_lse_merge(const float* o_part, const float* lse_part, void* o, float* lse,
-                             int B, int H, int S, int d, void* stream) {
+}  // extern "C"
+
+namespace {
+attn_status_t launch_merge(const float* o_part, const float* lse_part, void* o, float* lse,
+                           int B, int H, int S, int R, int d, void* stream) {
     if (!o_part || !lse_part || !o || !lse) return ATTN_ERR_INVALID_ARG;
     attn_status_t s = check_sizes(B, H, 1, 1);
     if (s != ATTN_OK) return s;
-    if (S < 1 || S > 65535) return ATTN_ERR_INVALID_ARG;
+    if (S < 1 || S > 65535 || R < 1 || R > 65535) return ATTN_ERR_INVALID_ARG;
+    if ((long long)S * R > (1ll << 24)) return ATTN_ERR_INVALID_ARG;
     if (d != 64 && d != 128) return ATTN_ERR_UNSUPPORTED;
     if (!aligned(o_part, 4) || !aligned(lse_part, 4) || !aligned(o, 2) || !aligned(lse, 4))
         return ATTN_ERR_ALIGNMENT;
     const int BH = B * H;
+    if ((long long)BH * S * R * d >= (1ll << 46)) return ATTN_ERR_INVALID_ARG;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    if (d == 128)
-        attn_lse_merge_kernel<128><<<BH, 128, 0, st>>>(o_part, lse_part,
-                                                       static_cast<uint16_t*>(o), lse, S);
-    else
-        attn_lse_merge_kernel<64><<<BH, 64, 0, st>>>(o_part, lse_part,
-                                                     static_cast<uint16_t*>(o), lse, S);
+    uint16_t* ob = static_cast<uint16_t*>(o);
+    const bool vec = aligned(o_part, 16);
+    if (d == 128) {
+        if (vec)
+            attn_lse_merge_kernel<128, true><<<BH, kMergeThreads, 0, st>>>(o_part, lse_part, ob,
+                                                                          lse, S, R, BH);
+        else
+            attn_lse_merge_kernel<128, false><<<BH, kMergeThreads, 0, st>>>(o_part, lse_part, ob,
+                                                                           lse, S, R, BH);
+    } else {
+        if (vec)
+            attn_lse_merge_kernel<64, true><<<BH, kMergeThreads, 0, st>>>(o_part, lse_part, ob,
+                                                                         lse, S, R, BH);
+        else
+            attn_lse_merge_kernel<64, false><<<BH, kMergeThreads, 0, st>>>(o_part, lse_part, ob,
+                                                                          lse, S, R, BH);
+    }
     return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+}  // namespace
+
+extern "C" {
+
+attn_status_t attn_lse_merge(const float* o_part, const float* lse_part, void* o, float* lse,
+                             int B, int H, int S, int d, void* stream) {
+    return launch_merge(o_part, lse_part, o, lse, B, H, S, 1, d, stream);
+}
+
+attn_status_t attn_lse_merge_gathered(const float* o_part, const float* lse_part, void* o,
+                                      float* lse, int R, int B, int H, int S, int d,
+                                      void* stream) {
+    return launch_merge(o_part, lse_part, o, lse, B, H, S, R, d, stream);
 }
 
 size_t attn_decode_workspace_bytes(int B, int H, int d, int num_splits) {

@@ -343,32 +343,98 @@ __global__ void __launch_bounds__(256, PAGED ? 4 : 1)
 }
 
 // ------------------------------------------------------------------ merge --
-// One block of D threads per (batch, head): thread x owns output column x.
+// One block of kMergeThreads per (batch, head):
 //   M = max_c lse_c;  w_c = exp(lse_c - M);  LSE = M + ln sum_c w_c;
 //   O = sum_c w_c O_c / sum_c w_c.
-template <int D>
-__global__ void __launch_bounds__(D)
+// The chunks may come from R groups (the KV shards of R GPUs, gathered one
+// after another): chunk s of group r of row bh is at ((r * BH + bh) * S + s),
+// which for R = 1 is the plain [BH, S] layout of attn_decode_partials.
+// Each thread owns 4 output columns of one chunk slot: D / 4 threads read one
+// partial row as one coalesced run of 16-byte loads, and the block covers
+// kMergeThreads / (D / 4) chunks per pass; the slots' sums are then added in
+// a fixed order through shared memory, so the result is deterministic.
+// VEC: o_part is 16-byte aligned (one 16-byte load per thread and chunk);
+// otherwise four 4-byte loads.
+constexpr int kMergeThreads = 256;
+
+template <bool VEC>
+__device__ __forceinline__ float4 load_f32x4(const float* p) {
+    if constexpr (VEC) return *reinterpret_cast<const float4*>(p);
+    return make_float4(p[0], p[1], p[2], p[3]);
+}
+
+template <int D, bool VEC>
+__global__ void __launch_bounds__(kMergeThreads)
     attn_lse_merge_kernel(const float* __restrict__ o_part, const float* __restrict__ lse_part,
-                          uint16_t* __restrict__ o, float* __restrict__ lse, int S) {
+                          uint16_t* __restrict__ o, float* __restrict__ lse, int S, int R,
+                          int BH) {
+    constexpr int kColThreads = D / 4;                       // threads per partial row
+    constexpr int kSlots = kMergeThreads / kColThreads;      // chunks per pass
+    __shared__ float s_red[kMergeThreads / 32];
+    __shared__ float4 s_acc[kSlots][kColThreads];
+    __shared__ float s_w[kSlots];
     const int bh = blockIdx.x;
-    const int x = threadIdx.x;
-    const float* lp = lse_part + (size_t)bh * S;
-    const float* op = o_part + (size_t)bh * S * D + x;
+    const int tid = threadIdx.x;
+    const int C = S * R;
+    // chunk c (0 <= c < C) of this row: group c / S, chunk c % S within it
+    auto row_of = [&](int c) -> size_t {
+        const int r = c / S;
+        return ((size_t)r * BH + bh) * S + (c - r * S);
+    };
+    // ---- M = max_c lse_c
     float M = -INFINITY;
-    for (int c = 0; c < S; ++c) M = fmaxf(M, lp[c]);
-    float W = 0.f, acc = 0.f;
+    for (int c = tid; c < C; c += kMergeThreads) M = fmaxf(M, lse_part[row_of(c)]);
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
+    if ((tid & 31) == 0) s_red[tid >> 5] = M;
+    __syncthreads();
+    M = s_red[0];
+#pragma unroll
+    for (int w = 1; w < kMergeThreads / 32; ++w) M = fmaxf(M, s_red[w]);
+    // ---- weighted sums, one chunk slot per group of kColThreads threads
+    const int slot = tid / kColThreads, col = tid % kColThreads;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    float W = 0.f;
     if (M != -INFINITY) {
         constexpr float kLog2e = 1.4426950408889634f;
-        for (int c = 0; c < S; ++c) {
-            const float w = fast_exp2((lp[c] - M) * kLog2e);
+        for (int c = slot; c < C; c += kSlots) {
+            const size_t row = row_of(c);
+            const float w = fast_exp2((lse_part[row] - M) * kLog2e);
+            const float4 x = load_f32x4<VEC>(o_part + row * D + 4 * col);
             W += w;
-            acc = fmaf(w, op[(size_t)c * D], acc);
+            acc.x = fmaf(w, x.x, acc.x);
+            acc.y = fmaf(w, x.y, acc.y);
+            acc.z = fmaf(w, x.z, acc.z);
+            acc.w = fmaf(w, x.w, acc.w);
         }
     }
-    const float out = W > 0.f ? acc / W : 0.f;
-    const uint32_t packed = pack_bf16x2(out, 0.f);
-    o[(size_t)bh * D + x] = (uint16_t)(packed & 0xFFFFu);
-    if (x == 0) lse[bh] = W > 0.f ? M + logf(W) : -INFINITY;
+    s_acc[slot][col] = acc;
+    if (col == 0) s_w[slot] = W;
+    __syncthreads();
+    // ---- add the slots in order; threads 0 .. kColThreads-1 write the row
+    if (tid < kColThreads) {
+        float4 t = s_acc[0][tid];
+        float Wt = s_w[0];
+#pragma unroll
+        for (int k = 1; k < kSlots; ++k) {
+            const float4 u = s_acc[k][tid];
+            t.x += u.x; t.y += u.y; t.z += u.z; t.w += u.w;
+            Wt += s_w[k];
+        }
+        const bool any = Wt > 0.f;
+        const uint32_t lo = pack_bf16x2(any ? t.x / Wt : 0.f, any ? t.y / Wt : 0.f);
+        const uint32_t hi = pack_bf16x2(any ? t.z / Wt : 0.f, any ? t.w / Wt : 0.f);
+        uint16_t* dst = o + (size_t)bh * D + 4 * tid;
+        if ((reinterpret_cast<uintptr_t>(dst) & 7) == 0) {
+            *reinterpret_cast<uint2*>(dst) = make_uint2(lo, hi);
+        } else {   // o is only required to be 2-byte aligned
+            dst[0] = (uint16_t)(lo & 0xFFFFu);
+            dst[1] = (uint16_t)(lo >> 16);
+            dst[2] = (uint16_t)(hi & 0xFFFFu);
+            dst[3] = (uint16_t)(hi >> 16);
+        }
+        if (tid == 0) lse[bh] = Wt > 0.f ? M + logf(Wt) : -INFINITY;
+    }
 }
 
 }  // namespace eattn

@@ -143,6 +143,26 @@ attn_status_t attn_lse_merge(const float *o_part, const float *lse_part, void *o
                              int B, int H, int S, int d, void *stream);
 
 /*
+ * Split-KV decode across GPUs, step 2: the same merge over partials gathered
+ * from R ranks, each of which computed S chunks of its own slice of the KV
+ * sequence (the decode split of mantramindai, "Follow-up questions to expect",
+ * last question, carried from thread blocks to GPUs: every rank holds a
+ * contiguous shard of the keys, runs attn_decode_partials on it, and the
+ * ranks' partials are all-gathered, rank after rank, into one buffer).
+ *
+ *   o_part   fp32 [R, B, H, S, d]   (read; rank r's attn_decode_partials output
+ *                                    at offset r * B * H * S * d)
+ *   lse_part fp32 [R, B, H, S]      (read)
+ *   o        bf16 [B, H, 1, d], lse fp32 [B, H, 1]   (written)
+ *   d in {64, 128}; 1 <= S, R <= 65535; S * R <= 2^24. The result does not
+ *   depend on how the keys were split (up to rounding); empty chunks (lse =
+ *   -inf) have weight 0. With R = 1 this is attn_lse_merge.
+ */
+attn_status_t attn_lse_merge_gathered(const float *o_part, const float *lse_part, void *o,
+                                      float *lse, int R, int B, int H, int S, int d,
+                                      void *stream);
+
+/*
  * Bytes of caller-provided workspace attn_decode_splitkv needs for the
  * partials: B*H*num_splits*(d + 1)*4, rounded up to 256. Returns 0 for
  * invalid sizes.

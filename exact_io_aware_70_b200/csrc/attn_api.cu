@@ -9,6 +9,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <atomic>
 #include <cmath>
 #include <cstdint>
 #include <cstring>
@@ -119,9 +120,26 @@ int current_device() {
     return dev;
 }
 
+// Unit-queue entry of the next forward launch (round robin): two launches
+// share an entry only if kFwdQueueSlots further launches are started while
+// the first is still running.
+std::atomic<unsigned> g_fwd_queue_rr{0};
+
+// Heads per group of the forward's unit order: as many heads as keep their
+// K and V within kFwdGroupBytes, so the CTAs in flight find them in L2.
+#ifndef EATTN_FWD_GROUP_BYTES
+#define EATTN_FWD_GROUP_BYTES (32ll << 20)
+#endif
+int fwd_group_heads(int BH, int Nkv, int d, int elem_bytes) {
+    const long long per_head = 2ll * Nkv * d * elem_bytes;
+    long long g = EATTN_FWD_GROUP_BYTES / (per_head > 0 ? per_head : 1);
+    if (g < 1) g = 1;
+    return g < BH ? (int)g : BH;
+}
+
 template <int D, bool CAUSAL, bool FP8 = false>
 attn_status_t launch_fwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                         const FwdParams& p, cudaStream_t stream) {
+                         FwdParams p, cudaStream_t stream) {
     using T = FwdTraits<D, FP8>;
     const int dev = current_device();
     if (dev < 0 || dev >= 64) return ATTN_ERR_CUDA;
@@ -143,6 +161,8 @@ attn_status_t launch_fwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUt
         sms = di.sms;
     }
     const int grid = p.num_units < sms ? p.num_units : sms;
+    p.group_heads = fwd_group_heads(p.BH, p.Nkv, D, T::kElemBytes);
+    p.queue_slot = (int)(g_fwd_queue_rr.fetch_add(1, std::memory_order_relaxed) % kFwdQueueSlots);
     kern<<<grid, T::kThreads, T::kSmemBytes, stream>>>(tq, tk, tv, p);
     return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }

@@ -86,6 +86,8 @@ struct FwdParams {
     int Nq, Nkv;
     int num_qb;         // ceil(Nq / 256)
     int num_units;      // BH * num_qb
+    int group_heads;    // heads per group of the unit order (see fwd_unit)
+    int queue_slot;     // which entry of g_fwd_queues this launch counts its units in
     float scale_log2;   // scale * log2(e)
 };
 
@@ -149,12 +151,23 @@ struct FwdTraits {
     static constexpr int kOtherRegs = 120;
     static_assert(2 * 128 * kSoftmaxRegs + 128 * kOtherRegs <= kThreads * kLaunchRegs,
                   "register split exceeds the launch allocation");
-    static constexpr int kNumBars = 2 * kSlots + 15;   // FwdBars<kSlots>::kCount
-    static constexpr int kSmemBytes = 1024 + (2 + kSlots) * kTileBytes + kNumBars * 8 + 16;
+    static constexpr int kNumBars = 2 * kSlots + 23;   // FwdBars<kSlots>::kCount
+    // epilogue staging: one 32-row x 64-byte (32 bf16 columns) block per softmax warp
+    static constexpr int kStageWarpBytes = 32 * 64;
+    static constexpr int kStageBytes = 8 * kStageWarpBytes;
+    static constexpr int kSmemBytes =
+        1024 + (2 + kSlots) * kTileBytes + kStageBytes + kNumBars * 8 + 16 + 16;
     static_assert(kSmemBytes <= 232448, "shared memory per CTA");
     static constexpr uint32_t kTmemCols = 512;
+    // Score buffers of 128 fp32 columns. With two (head dim 128: 2 x 128 + 2 x
+    // 128 O columns fill the 512) tile t always uses buffer t, so S_t(j+1) can
+    // only be computed once P_t(j) V has been issued (it overwrites P_t(j)).
+    // With three (head dim 64: 3 x 128 + 2 x 64 = 512) the S products rotate
+    // over the buffers in issue order and S_t(j+1) is computed ahead, while
+    // the softmax still works on S_t(j) (see fwd_mma).
+    static constexpr int kSBufs = (3 * 128 + 2 * D <= 512) ? 3 : 2;
     static constexpr uint32_t kColS0 = 0, kColS1 = 128;
-    static constexpr uint32_t kColO0 = 256, kColO1 = 256 + D;
+    static constexpr uint32_t kColO0 = 128 * kSBufs, kColO1 = 128 * kSBufs + D;
 };
 
 // One exponent pair in every kPolyEvery<D, FP8> goes to the FMA-pipe polynomial
@@ -176,15 +189,26 @@ template <int D, bool FP8 = false>
 constexpr int kPolyEvery =
     FP8 ? EATTN_POLY_EVERY_FP8 : ((D == 128) ? EATTN_POLY_EVERY_D128 : EATTN_POLY_EVERY_D64);
 
-// Unit handled by this CTA in round r (snake order), or -1 past the end.
-__device__ __forceinline__ int fwd_unit_of_round(int r, int num_units) {
-    const int g = gridDim.x, i = blockIdx.x;
-    const long long u = (long long)r * g + ((r & 1) ? (g - 1 - i) : i);
-    return u < num_units ? (int)u : -1;
+// Work units are handed out dynamically: each CTA's producer takes the next
+// index from a device counter (p.queue[0], one atomicAdd per unit) and passes
+// it to the MMA and softmax roles through a two-entry ring in shared memory.
+// Index u maps to a unit in this order: the heads are taken in groups of
+// p.group_heads (the host sizes a group so that its K and V fit comfortably
+// in L2), and inside a group the query blocks go heaviest first (latest block
+// first under the causal mask), the group's heads interleaved. So the CTAs in
+// flight share the K/V tiles of a few heads, which stay in L2 instead of being
+// re-read from DRAM, and each group ends with its lightest units, which keeps
+// the SMs balanced as a longest-first schedule would.
+// g_fwd_queues[2 * slot] counts units handed out, g_fwd_queues[2 * slot + 1]
+// the CTAs that have finished; both are zero when a launch starts, and the
+// launch's last CTA sets them back to zero.
+constexpr int kFwdQueueSlots = 64;
+__device__ int g_fwd_queues[2 * kFwdQueueSlots];
+
+__device__ __forceinline__ int fwd_fetch_unit(const FwdParams& p) {
+    const int u = atomicAdd(&g_fwd_queues[2 * p.queue_slot], 1);
+    return u < p.num_units ? u : -1;
 }
-#define FWD_FOR_EACH_UNIT(u, p)                                                   \
-    for (int round_ = 0, u = 0; (long long)round_ * gridDim.x < (p).num_units; ++round_) \
-        if ((u = fwd_unit_of_round(round_, (p).num_units)) >= 0)
 
 struct FwdUnit {
     int bh, qb;
@@ -195,8 +219,12 @@ struct FwdUnit {
 template <bool CAUSAL>
 __device__ __forceinline__ FwdUnit fwd_unit(int u, const FwdParams& p) {
     FwdUnit x;
-    x.qb = p.num_qb - 1 - u / p.BH;   // heaviest (latest) query blocks first
-    x.bh = u % p.BH;
+    const int per_group = p.group_heads * p.num_qb;
+    const int g = u / per_group;
+    const int r = u - g * per_group;
+    const int heads = min(p.group_heads, p.BH - g * p.group_heads);   // the last group may be short
+    x.qb = p.num_qb - 1 - r / heads;   // heaviest (latest) query blocks first
+    x.bh = g * p.group_heads + r % heads;
 #pragma unroll
     for (int t = 0; t < 2; ++t) {
         const long long r0 = (long long)x.qb * 256 + t * 128;
@@ -215,10 +243,18 @@ __device__ __forceinline__ FwdUnit fwd_unit(int u, const FwdParams& p) {
     return x;
 }
 
+// Position of S_t(i) among the unit's score products in issue order: all
+// products of index i' < i (tile 0's before tile 1's at each index), then
+// S_0(i) before S_1(i).
+__device__ __forceinline__ int fwd_s_pos(const FwdUnit& x, int t, int i) {
+    return min(i, x.n[0]) + min(i, x.n[1]) + ((t == 1 && i < x.n[0]) ? 1 : 0);
+}
+
 // mbarrier addresses, all derived from one shared-memory base address so that
 // only a single register is live across the roles. Layout (8 bytes each):
 // kv_full[S], kv_empty[S], then 2 each of q_full, q_empty, s_full, p_lo, p_hi,
-// o_final, o_free, then drain.
+// o_final, o_free, then drain, then 2 each of unit_full, unit_empty, s_full_b,
+// pv_done.
 template <int S>
 struct FwdBars {
     uint32_t base;
@@ -232,8 +268,46 @@ struct FwdBars {
     __device__ __forceinline__ uint32_t o_final(int t) const { return base + 8 * (2 * S + 10 + t); }
     __device__ __forceinline__ uint32_t o_free(int t) const { return base + 8 * (2 * S + 12 + t); }
     __device__ __forceinline__ uint32_t drain() const { return base + 8 * (2 * S + 14); }
-    static constexpr int kCount = 2 * S + 15;
+    __device__ __forceinline__ uint32_t unit_full(int i) const { return base + 8 * (2 * S + 15 + i); }
+    __device__ __forceinline__ uint32_t unit_empty(int i) const { return base + 8 * (2 * S + 17 + i); }
+    // three score buffers only: S_t products alternate between s_full(t) and
+    // s_full_b(t) (one may complete before the softmax has seen the other);
+    // pv_done(t) completes with every P_t V product
+    __device__ __forceinline__ uint32_t s_full_b(int t) const { return base + 8 * (2 * S + 19 + t); }
+    __device__ __forceinline__ uint32_t pv_done(int t) const { return base + 8 * (2 * S + 21 + t); }
+    // barrier and parity of tile t's c-th score product (c counted over the CTA's life)
+    template <int kSBufs>
+    __device__ __forceinline__ uint32_t s_bar(int t, uint32_t c) const {
+        return (kSBufs == 3 && (c & 1)) ? s_full_b(t) : s_full(t);
+    }
+    template <int kSBufs>
+    static __device__ __forceinline__ uint32_t s_parity(uint32_t c) {
+        return kSBufs == 3 ? (c >> 1) & 1 : c & 1;
+    }
+    static constexpr int kCount = 2 * S + 23;
+    // shared-memory words after the barriers: TMEM base, abort flag, unit ring[2]
+    __device__ __forceinline__ volatile int* unit_slot(int i) const {
+        return reinterpret_cast<volatile int*>(unit_ring_ptr) + i;
+    }
+    uint8_t* unit_ring_ptr;
 };
+
+// Readers of a unit-ring entry: the MMA issuer and one lane of each of the 8
+// softmax warps.
+constexpr int kUnitReaders = 9;
+
+// Next unit for a consumer role: waits for ring entry k, reads it and
+// releases the entry (the MMA issuer and lane 0 of each softmax warp count as
+// its readers). Returns false on a failed wait; *u = -1 marks the end.
+template <int S>
+__device__ __forceinline__ bool fwd_next_unit(const FwdBars<S>& b, uint32_t k, bool arrive,
+                                              volatile int* abort_flag, int* u) {
+    const int slot = k & 1;
+    if (!mbar_wait(b.unit_full(slot), (k >> 1) & 1, abort_flag, &g_attn_status)) return false;
+    *u = *b.unit_slot(slot);
+    if (arrive) mbar_arrive(b.unit_empty(slot));
+    return true;
+}
 
 // Bounded wait executed by a whole warp; the outcome is made warp-uniform.
 __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag) {
@@ -267,7 +341,14 @@ __device__ void fwd_producer(const FwdParams& p, const CUtensorMap* tq, const CU
     const uint64_t pol_kv = l2_policy_evict_last();
     uint32_t kv_iter = 0;
     uint32_t q_issued[2] = {0, 0};
-    FWD_FOR_EACH_UNIT(u, p) {
+    int u = fwd_fetch_unit(p);
+    for (uint32_t k = 0;; ++k) {
+        // publish unit u (or the end) in ring entry k once its last readers are done
+        const int slot = k & 1;
+        if (k >= 2 && !role_wait(b.unit_empty(slot), ((k >> 1) - 1) & 1, abort_flag)) goto fail;
+        *b.unit_slot(slot) = u;
+        mbar_arrive(b.unit_full(slot));
+        if (u < 0) break;
         const FwdUnit x = fwd_unit<CAUSAL>(u, p);
         for (int t = 0; t < 2; ++t) {
             if (q_issued[t] > 0 && !role_wait(b.q_empty(t), (q_issued[t] - 1) & 1, abort_flag))
@@ -284,6 +365,7 @@ __device__ void fwd_producer(const FwdParams& p, const CUtensorMap* tq, const CU
                                   pn * T::kPanelElems, x.qb * 256 + t * 128, x.bh, leader);
             ++q_issued[t];
         }
+        u = fwd_fetch_unit(p);   // the next unit, fetched while this one's tiles stream in
         for (int j = 0; j < x.nmax; ++j) {
 #pragma unroll
             for (int which = 0; which < 2; ++which) {   // K_j, then V_j
@@ -378,6 +460,113 @@ __device__ __forceinline__ void fwd_issue_pv(uint32_t tmem_o, uint32_t tmem_p, u
     }
 }
 
+// Three score buffers (head dim 64). Per K/V step j the issue order is
+//   S_0(j+1), P_0(j) V_j, S_1(j+1), P_1(j) V_j,
+// every score product going to buffer (products issued so far) mod 3. The
+// buffer S_t(j+1) overwrites last held the product issued three before it,
+// whose P V has always been issued by then (S_1(j) at the end of step j-1 for
+// S_0(j+1); S_0(j) just before for S_1(j+1); earlier still when a tile has
+// fewer steps, and all of the previous unit's), and tensor-core operations
+// run in issue order. So S_t(j+1) is computed while the softmax group still
+// works on S_t(j), and the group finds it ready when it hands over P_t(j).
+template <int D, bool CAUSAL, bool FP8>
+__device__ void fwd_mma_ahead(const FwdParams& p, uint32_t tbase, uint32_t sQ, uint32_t sKV,
+                              const FwdBars<FwdTraits<D, FP8>::kSlots>& b, uint32_t leader,
+                              volatile int* abort_flag) {
+    using T = FwdTraits<D, FP8>;
+    static_assert(T::kSBufs == 3, "three score buffers");
+    static_assert(!EATTN_SPLIT_P, "P is handed over once per step here");
+    constexpr uint64_t kTileStep = T::kTileBytes >> 4;
+    const uint64_t dq0 = fwd_sdesc<T>(sQ, 16);
+    const uint64_t dk0 = fwd_sdesc<T>(sKV, 16);                       // K-major K tile
+    const uint64_t dv0 = fwd_sdesc<T>(sKV, T::kPanelBytes);           // MN-major V tile
+    const uint32_t colO[2] = {T::kColO0, T::kColO1};
+    uint32_t kv_iter = 0, q_use = 0, s_issued = 0;
+    uint32_t o_use[2] = {0, 0}, p_cnt[2] = {0, 0}, s_cnt[2] = {0, 0};
+    uint32_t cur_col[2] = {0, 0};   // buffer holding S_t(j) / P_t(j)
+    for (uint32_t k = 0;; ++k) {
+        int u;
+        if (!fwd_next_unit(b, k, true, abort_flag, &u)) goto done;
+        if (u < 0) break;
+        {
+            const FwdUnit x = fwd_unit<CAUSAL>(u, p);
+            if (!role_wait(b.q_full(0), q_use & 1, abort_flag)) goto done;
+            if (!role_wait(b.q_full(1), q_use & 1, abort_flag)) goto done;
+            tc_fence_after_sync();
+            // S_t(i) into the next buffer in rotation; Q_t is released after its last product
+            auto issue_s = [&](int t, int i, uint32_t kslot) {
+                const uint32_t col = (s_issued++ % 3) * 128;
+                fwd_issue_s<D, FP8>(tbase + col, dq0 + t * kTileStep, dk0 + kslot * kTileStep,
+                                    leader);
+                mma_commit_w(b.template s_bar<3>(t, s_cnt[t]++), leader);
+                if (i == x.n[t] - 1) mma_commit_w(b.q_empty(t), leader);
+                return col;
+            };
+            if (x.nmax > 0) {
+                uint32_t kslot = kv_iter % T::kSlots;
+                if (!role_wait(b.kv_full(kslot), (kv_iter / T::kSlots) & 1, abort_flag)) goto done;
+                tc_fence_after_sync();
+                for (int t = 0; t < 2; ++t)
+                    if (x.n[t] > 0) cur_col[t] = issue_s(t, 0, kslot);
+                mma_commit_w(b.kv_empty(kslot), leader);
+                ++kv_iter;
+                for (int j = 0; j < x.nmax; ++j) {
+                    const uint32_t vslot = kv_iter % T::kSlots;   // V_j arrived with K_j
+                    ++kv_iter;
+                    const bool has_next = j + 1 < x.nmax;
+                    kslot = kv_iter % T::kSlots;
+                    if (has_next) {
+                        if (!role_wait(b.kv_full(kslot), (kv_iter / T::kSlots) & 1, abort_flag))
+                            goto done;
+                        tc_fence_after_sync();
+                    }
+                    for (int t = 0; t < 2; ++t) {
+                        uint32_t next_col = cur_col[t];
+                        if (j + 1 < x.n[t]) next_col = issue_s(t, j + 1, kslot);
+                        if (j < x.n[t]) {
+                            // P_t hand-overs alternate between two barriers: the group may
+                            // release P_t(j+1) before this wait for P_t(j) has run, since
+                            // S_t(j+1) is already issued; P_t(j+2) it may not.
+                            if (!role_wait((p_cnt[t] & 1) ? b.p_lo(t) : b.p_hi(t),
+                                           (p_cnt[t] >> 1) & 1, abort_flag))
+                                goto done;
+                            ++p_cnt[t];
+                            if (j == 0 && o_use[t] > 0 &&
+                                !role_wait(b.o_free(t), (o_use[t] - 1) & 1, abort_flag))
+                                goto done;
+                            tc_fence_after_sync();
+                            fwd_issue_pv<D, FP8>(tbase + colO[t], tbase + cur_col[t],
+                                                 dv0 + vslot * kTileStep, j > 0, 0, leader);
+                            fwd_issue_pv<D, FP8>(tbase + colO[t], tbase + cur_col[t],
+                                                 dv0 + vslot * kTileStep, true, 1, leader);
+                            mma_commit_w(b.pv_done(t), leader);
+                            if (j == x.n[t] - 1) mma_commit_w(b.o_final(t), leader);
+                        }
+                        cur_col[t] = next_col;
+                    }
+                    mma_commit_w(b.kv_empty(vslot), leader);
+                    if (has_next) {
+                        mma_commit_w(b.kv_empty(kslot), leader);
+                        ++kv_iter;
+                    }
+                }
+            }
+            // Q tiles without any S product in this unit are released here
+            for (int t = 0; t < 2; ++t)
+                if (x.n[t] == 0) mma_commit_w(b.q_empty(t), leader);
+            ++q_use;
+            for (int t = 0; t < 2; ++t)
+                if (x.n[t] > 0) ++o_use[t];
+        }
+    }
+done: {
+    // Every MMA issued so far must finish before tensor memory is released.
+    volatile int no_abort = 0;
+    mma_commit_w(b.drain(), leader);
+    mbar_wait(b.drain(), 0, &no_abort, &g_attn_status);
+}
+}
+
 // Run by the whole MMA warp with converged control flow; lane 0 issues.
 template <int D, bool CAUSAL, bool FP8>
 __device__ void fwd_mma(const FwdParams& p, uint32_t tbase, uint32_t sQ, uint32_t sKV,
@@ -392,7 +581,10 @@ __device__ void fwd_mma(const FwdParams& p, uint32_t tbase, uint32_t sQ, uint32_
     const uint32_t colO[2] = {T::kColO0, T::kColO1};
     uint32_t kv_iter = 0, q_use = 0;
     uint32_t o_use[2] = {0, 0}, p_phase[2] = {0, 0};
-    FWD_FOR_EACH_UNIT(u, p) {
+    for (uint32_t k = 0;; ++k) {
+        int u;
+        if (!fwd_next_unit(b, k, true, abort_flag, &u)) goto done;
+        if (u < 0) break;
         const FwdUnit x = fwd_unit<CAUSAL>(u, p);
         if (!role_wait(b.q_full(0), q_use & 1, abort_flag)) goto done;
         if (!role_wait(b.q_full(1), q_use & 1, abort_flag)) goto done;
@@ -475,6 +667,37 @@ done: {
 }
 
 // --------------------------------------------------------------- softmax --
+// Epilogue store of one 32-column chunk of this warp's 32 rows. Lane l holds
+// row l's 32 bf16 values (w, 16 words). They go through the warp's 2 KB
+// staging block so that the global stores are row-contiguous: each store
+// instruction writes 8 rows x 64 bytes (4 lanes per row, 16 bytes each), i.e.
+// whole 32-byte sectors, instead of 32 rows x 16 bytes. In the staging block,
+// rows 2p and 2p+1 share a 128-byte line and row r's 16-byte piece k sits in
+// slot (r & 1) * 4 + (k ^ (p & 3)) of its line, so that neither the row-wise
+// writes nor the piece-wise reads have bank conflicts.
+__device__ __forceinline__ uint32_t stage_slot(int r, int k) {
+    const int pr = r >> 1;
+    return (uint32_t)((pr * 8 + (r & 1) * 4 + (k ^ (pr & 3))) * 16);
+}
+
+template <int D>
+__device__ __forceinline__ void fwd_store_chunk(uint32_t stage, const uint32_t (&w)[16], int lane,
+                                                uint16_t* o_rows, int c, int valid_rows) {
+    __syncwarp();   // the previous chunk's reads of the staging block are done
+#pragma unroll
+    for (int k = 0; k < 4; ++k)
+        st_shared_v4(stage + stage_slot(lane, k), w[4 * k], w[4 * k + 1], w[4 * k + 2],
+                     w[4 * k + 3]);
+    __syncwarp();
+#pragma unroll 1
+    for (int i = 0; i < 4; ++i) {
+        const int r = i * 8 + (lane >> 2), k = lane & 3;
+        const uint4 val = ld_shared_v4(stage + stage_slot(r, k));
+        if (r < valid_rows)
+            *reinterpret_cast<uint4*>(o_rows + (size_t)r * D + c + 8 * k) = val;
+    }
+}
+
 template <int D, bool CAUSAL, bool FP8>
 __device__ void fwd_softmax(const FwdParams& p, uint32_t tbase,
                             const FwdBars<FwdTraits<D, FP8>::kSlots>& b, int warp, int lane,
@@ -484,14 +707,20 @@ __device__ void fwd_softmax(const FwdParams& p, uint32_t tbase,
     const int quarter = warp & 3;            // TMEM lane quarter this warp may access
     const int r = quarter * 32 + lane;       // row within the tile = TMEM lane
     const uint32_t lane_off = uint32_t(quarter * 32) << 16;
-    const uint32_t tS = tbase + lane_off + (t ? T::kColS1 : T::kColS0);
     const uint32_t tO = tbase + lane_off + (t ? T::kColO1 : T::kColO0);
-    const uint32_t bar_s = b.s_full(t);
     const uint32_t bar_plo = b.p_lo(t), bar_phi = b.p_hi(t);
     const uint32_t bar_of = b.o_final(t), bar_ofree = b.o_free(t);
-    uint32_t s_phase = 0, o_use = 0;
+    uint32_t s_cnt = 0, o_use = 0;
+    uint32_t p_cnt = 0;       // P_t tiles handed over so far (= P_t V products issued or due)
+    uint32_t s_base = 0;      // score products issued in earlier units (three buffers)
 
-    FWD_FOR_EACH_UNIT(u, p) {
+    for (uint32_t k = 0;; ++k) {
+        int u;
+        const bool ok = fwd_next_unit(b, k, false, abort_flag, &u);
+        __syncwarp();
+        if (lane == 0 && ok) mbar_arrive(b.unit_empty(k & 1));
+        if (!__all_sync(0xffffffffu, ok)) return;
+        if (u < 0) break;
         const FwdUnit x = fwd_unit<CAUSAL>(u, p);
         // scores in log2 units; e4m3 inputs fold their Q and K factors in here
         const float c2 = FP8 ? p.scale_log2 * p.q_descale[x.bh] * p.k_descale[x.bh]
@@ -506,8 +735,15 @@ __device__ void fwd_softmax(const FwdParams& p, uint32_t tbase,
         float l = 0.f;              // running sum of 2^(s*c2 - m_ref)
 
         for (int j = 0; j < n; ++j) {
-            if (!warp_wait(bar_s, s_phase, abort_flag)) return;
-            s_phase ^= 1;
+            // the TMEM columns holding S_t(j), and then P_t(j)
+            const uint32_t tS =
+                tbase + lane_off +
+                (T::kSBufs == 3 ? ((s_base + fwd_s_pos(x, t, j)) % 3) * 128
+                                : (t ? T::kColS1 : T::kColS0));
+            if (!warp_wait(b.template s_bar<T::kSBufs>(t, s_cnt),
+                           FwdBars<T::kSlots>::template s_parity<T::kSBufs>(s_cnt), abort_flag))
+                return;
+            ++s_cnt;
             tc_fence_after_sync();
             uint32_t sr[128];
             tmem_ld128(tS, sr);
@@ -573,8 +809,15 @@ __device__ void fwd_softmax(const FwdParams& p, uint32_t tbase,
                 }
                 if (h == 0 && any_need && j > 0) {
                     // Rescale O_t by alpha (1 for rows whose max did not move)
-                    // before any of P_t(j) V is released. O_t is stable here: the
-                    // commit that signalled S_t(j) also covers P_t(j-1) V.
+                    // before any of P_t(j) V is released. O_t must hold P_t(j-1) V:
+                    // with two score buffers the commit that signalled S_t(j)
+                    // covers it; with three, S_t(j) was issued before it, so wait
+                    // for its own completion (P_t(j) is not released yet, so that
+                    // barrier cannot be a phase further on).
+                    if (T::kSBufs == 3 &&
+                        !warp_wait(b.pv_done(t), (p_cnt - 1) & 1, abort_flag))
+                        return;
+                    tc_fence_after_sync();
 #pragma unroll
                     for (int c = 0; c < D; c += 32) {
                         uint32_t orr[32];
@@ -593,15 +836,19 @@ __device__ void fwd_softmax(const FwdParams& p, uint32_t tbase,
                 if (EATTN_SPLIT_P || h == 1) {
                     tmem_wait_st();
                     tc_fence_before_sync();
-                    mbar_arrive(h == 0 ? bar_plo : bar_phi);
+                    // three score buffers: P_t tiles alternate between p_hi and p_lo
+                    mbar_arrive(T::kSBufs == 3 ? ((p_cnt & 1) ? bar_plo : bar_phi)
+                                               : (h == 0 ? bar_plo : bar_phi));
                 }
             }
+            ++p_cnt;
             float la0, la1, lb0, lb1;
             f2_unpack(lsum_a, la0, la1);
             f2_unpack(lsum_b, lb0, lb1);
             l = l * alpha + ((la0 + la1) + (lb0 + lb1));
         }
 
+        s_base += x.n[0] + x.n[1];
         uint16_t* orow = p.o + ((size_t)x.bh * p.Nq + (size_t)(row_valid ? qrow : 0)) * D;
         // A row that sees no key at all (causal with Nq > Nkv) is O = 0, LSE = -inf by
         // definition; its polynomial exponentials of -inf scores are tiny, not zero.
@@ -610,7 +857,13 @@ __device__ void fwd_softmax(const FwdParams& p, uint32_t tbase,
             if (!warp_wait(bar_of, o_use & 1, abort_flag)) return;
             tc_fence_after_sync();
             const float inv = l > 0.f ? (FP8 ? p.v_descale[x.bh] : 1.0f) / l : 0.f;
-#pragma unroll
+            // this warp's 32 rows: the first one and how many of them exist
+            const int row0 = x.qb * 256 + t * 128 + quarter * 32;
+            const int valid_rows = min(32, p.Nq - row0);
+            uint16_t* o_rows = p.o + ((size_t)x.bh * p.Nq + (size_t)max(row0, 0)) * D;
+            // the staging blocks sit right below the barriers
+            const uint32_t stage = b.base - T::kStageBytes + warp * T::kStageWarpBytes;
+#pragma unroll 1
             for (int c = 0; c < D; c += 32) {
                 uint32_t orr[32];
                 tmem_ld32(tO + c, orr);
@@ -620,12 +873,7 @@ __device__ void fwd_softmax(const FwdParams& p, uint32_t tbase,
                 for (int i = 0; i < 16; ++i)
                     w[i] = pack_bf16x2(__uint_as_float(orr[2 * i]) * inv,
                                        __uint_as_float(orr[2 * i + 1]) * inv);
-                if (row_valid) {
-                    uint4* dst = reinterpret_cast<uint4*>(orow + c);
-#pragma unroll
-                    for (int k = 0; k < 4; ++k)
-                        dst[k] = make_uint4(w[4 * k], w[4 * k + 1], w[4 * k + 2], w[4 * k + 3]);
-                }
+                fwd_store_chunk<D>(stage, w, lane, o_rows, c, valid_rows);
             }
             tc_fence_before_sync();
             mbar_arrive(bar_ofree);
@@ -653,12 +901,15 @@ __global__ void __launch_bounds__(384, 1)
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const uint32_t sQ = smem_addr(smem);
     const uint32_t sKV = sQ + 2 * T::kTileBytes;
-    uint8_t* bar_ptr = smem + (2 + T::kSlots) * T::kTileBytes;
+    // epilogue staging blocks, then the barriers (fwd_softmax finds its block
+    // kStageBytes below the barrier base)
+    uint8_t* bar_ptr = smem + (2 + T::kSlots) * T::kTileBytes + T::kStageBytes;
     const uint32_t bar0 = smem_addr(bar_ptr);
     FwdBars<T::kSlots> b;
     b.base = bar0;
     uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bar_ptr + 8 * FwdBars<T::kSlots>::kCount);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
+    b.unit_ring_ptr = reinterpret_cast<uint8_t*>(tmem_holder + 2);
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -678,6 +929,12 @@ __global__ void __launch_bounds__(384, 1)
             mbar_init(b.o_free(t), 128);
         }
         mbar_init(b.drain(), 1);
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(b.unit_full(i), 1);
+            mbar_init(b.unit_empty(i), kUnitReaders);
+            mbar_init(b.s_full_b(i), 1);
+            mbar_init(b.pv_done(i), 1);
+        }
         *abort_flag = 0;
         fence_mbar_init();
     }
@@ -703,8 +960,12 @@ __global__ void __launch_bounds__(384, 1)
         const bool issuer_thread = EATTN_WARP_ISSUE ? true : lane == 0;
         if (warp == 8 && issuer_thread)
             fwd_producer<D, CAUSAL, FP8>(p, &tm_q, &tm_k, &tm_v, sQ, sKV, b, lane == 0, abort_flag);
-        else if (warp == 9 && issuer_thread)
-            fwd_mma<D, CAUSAL, FP8>(p, tbase, sQ, sKV, b, lane == 0, abort_flag);
+        else if (warp == 9 && issuer_thread) {
+            if constexpr (T::kSBufs == 3)
+                fwd_mma_ahead<D, CAUSAL, FP8>(p, tbase, sQ, sKV, b, lane == 0, abort_flag);
+            else
+                fwd_mma<D, CAUSAL, FP8>(p, tbase, sQ, sKV, b, lane == 0, abort_flag);
+        }
     }
 
     tc_fence_before_sync();
@@ -713,6 +974,16 @@ __global__ void __launch_bounds__(384, 1)
     if (warp == 9) {
         __syncwarp();
         tmem_dealloc(tbase, T::kTmemCols);
+    }
+    // Every role of this CTA is done, so its producer has made its last fetch.
+    // The CTA that finishes last returns the queue to zero for the next launch.
+    if (threadIdx.x == 0) {
+        int* q = &g_fwd_queues[2 * p.queue_slot];
+        __threadfence();
+        if (atomicAdd(q + 1, 1) == (int)gridDim.x - 1) {
+            atomicExch(q, 0);
+            atomicExch(q + 1, 0);
+        }
     }
 }
 

@@ -86,3 +86,17 @@ def test_reference_arm_never_loads_the_cuda_library():
                          timeout=600, cwd=ROOT)
     assert out.returncode == 0, out.stderr[-2000:]
     assert "CLEAN" in out.stdout
+
+
+def test_oracle_sample_counts_flops_of_the_workload_it_samples():
+    """The per-workload CPU baseline counts causal and non-causal rows right."""
+    from seeded_inputs import WORKLOADS
+    tiny = bench.oracle_prefill_sample(0.05, max_heads=1, w=WORKLOADS["tiny"])
+    w = WORKLOADS["tiny"]                        # non-causal: every row sees all keys
+    assert tiny["flops"] == tiny["heads"] * tiny["rows"] * 4.0 * w.d * w.Nkv
+    g = WORKLOADS["gpt2_1k"]
+    s = bench.oracle_prefill_sample(0.05, max_rows=64, max_heads=1, w=g)
+    rows = np.linspace(0, g.Nq - 1, s["rows"]).astype(np.int64)
+    assert s["flops"] == s["heads"] * sum(4.0 * g.d * (int(r) + 1) for r in rows)
+    cb = bench.prefill_cpu_baseline(g, 0.05)
+    assert cb["kind"] == "oracle" and cb["cores"] >= 1 and cb["value"] > 0 and "gpt2_1k" in cb["sample"]

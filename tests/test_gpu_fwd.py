@@ -30,6 +30,10 @@ SWEEP = [
     (2, 1, 3000, 1000, 128, True),  # Nq > Nkv at length: 2000 rows per head see no key
     (8, 64, 100, 100, 128, False),  # 512 units: several persistent rounds, a partial last one
     (4, 100, 257, 257, 64, True),   # 800 units of two sizes over 5.4 rounds
+    # long K/V rows: the unit order groups the heads (3 heads of 10.7 MB of K/V
+    # per group, the last group short; then one head per group)
+    (2, 4, 300, 21845, 128, True),
+    (1, 3, 512, 65536, 128, False),
 ]
 
 
@@ -122,3 +126,29 @@ def test_deterministic():
     o1, l1 = gpu_util.run_fwd(q, k, v, True, 0.088)
     o2, l2 = gpu_util.run_fwd(q, k, v, True, 0.088)
     assert torch.equal(o1, o2) and torch.equal(l1, l2)
+
+
+def test_concurrent_launches_on_two_streams():
+    """Launches in flight at the same time on two streams take their work units
+    from different queue entries, so neither steals the other's units."""
+    from seeded_inputs import make_qkv
+    m = gpu_util.ea()
+    shapes = [(2, 8, 1000, 1000, 128, True, 41), (4, 6, 777, 777, 64, False, 42)]
+    ins, outs, streams = [], [], [torch.cuda.Stream(), torch.cuda.Stream()]
+    for (B, H, Nq, Nkv, d, causal, seed) in shapes:
+        q, k, v = (t.cuda() for t in make_qkv(B, H, Nq, Nkv, d, seed))
+        ins.append((q, k, v))
+        outs.append((torch.empty_like(q), torch.empty((B, H, Nq), dtype=torch.float32,
+                                                      device="cuda")))
+    torch.cuda.synchronize()
+    for rep in range(3):
+        for i, (B, H, Nq, Nkv, d, causal, seed) in enumerate(shapes):
+            q, k, v = ins[i]
+            o, lse = outs[i]
+            m.attn_fwd(q, k, v, o, lse, causal, float(np.float32(1 / np.sqrt(d))),
+                       stream=streams[i].cuda_stream)
+        torch.cuda.synchronize()
+        assert m.attn_status() == 0
+        for i, (B, H, Nq, Nkv, d, causal, seed) in enumerate(shapes):
+            ref_o, ref_l = gpu_util.run_fwd(*ins[i], causal, float(np.float32(1 / np.sqrt(d))))
+            assert torch.equal(outs[i][0], ref_o) and torch.equal(outs[i][1], ref_l), (rep, i)

@@ -12,6 +12,7 @@ Entry points (same names as the C ABI):
   attn_bwd_workspace_bytes(B, H, Nq, d)
   attn_decode_partials(q, k, v, o_part, lse_part, scale, num_splits)
   attn_lse_merge(o_part, lse_part, o, lse)
+  attn_lse_merge_gathered(o_part, lse_part, o, lse)  merge of partials gathered from R GPUs
   attn_decode_splitkv(q, k, v, o, lse, scale, num_splits, workspace)
   attn_decode_workspace_bytes(B, H, d, num_splits)
   attn_decode_paged(q, k_cache, v_cache, block_table, seq_lens, o, lse, scale, num_splits,
@@ -27,8 +28,9 @@ import ctypes
 import os
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-# EXACT_ATTN_LIB may name another build of the same library (e.g. one compiled
-# with different tuning macros); it must exist, there is no fallback either way.
+# EXACT_ATTN_LIB may name another build of the same library (e.g. the debug
+# build, libexact_attn_b200_debug.so, whose kernels check their indices); it
+# must exist, there is no fallback either way.
 LIB_PATH = os.environ.get("EXACT_ATTN_LIB") or os.path.join(_HERE, "libexact_attn_b200.so")
 
 if not os.path.exists(LIB_PATH):
@@ -81,6 +83,7 @@ ATTN_ERR_CUDA = 4
 ATTN_ERR_TIMEOUT = 5
 ATTN_ERR_SCRATCH_LIMIT = 6
 ATTN_ERR_BAD_INDEX = 7
+ATTN_ERR_INDEX_CHECK = 8   # debug build only: a kernel index check failed
 
 
 class AttnError(RuntimeError):

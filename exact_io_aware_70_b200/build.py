@@ -14,6 +14,9 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libexact_attn_b200.so")
+# The debug build: the same sources with -DATTN_DEBUG, whose kernels check the
+# global-memory indices they compute (see dcheck in csrc/ptx_sm100.cuh).
+LIB_DEBUG = os.path.join(HERE, "libexact_attn_b200_debug.so")
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 
 FLAGS = [
@@ -30,26 +33,28 @@ def sources():
             if f.endswith((".cu", ".cuh"))] + [os.path.join(ROOT, "include", "exact_attn.h")]
 
 
-def up_to_date() -> bool:
-    if not os.path.exists(LIB):
+def up_to_date(lib: str = LIB) -> bool:
+    if not os.path.exists(lib):
         return False
-    t = os.path.getmtime(LIB)
+    t = os.path.getmtime(lib)
     return all(os.path.getmtime(s) <= t for s in sources())
 
 
-def build(force: bool = False, verbose: bool = False) -> str:
-    if not force and up_to_date():
-        return LIB
-    cmd = [NVCC, *FLAGS, "-I", os.path.join(ROOT, "include"), "-I", CSRC,
-           os.path.join(CSRC, "attn_api.cu"), os.path.join(CSRC, "attn_noalloc.cu"), "-o", LIB]
+def build(force: bool = False, verbose: bool = False, debug: bool = False) -> str:
+    lib = LIB_DEBUG if debug else LIB
+    if not force and up_to_date(lib):
+        return lib
+    cmd = [NVCC, *FLAGS, *(["-DATTN_DEBUG"] if debug else []), "-I", os.path.join(ROOT, "include"),
+           "-I", CSRC, os.path.join(CSRC, "attn_api.cu"), os.path.join(CSRC, "attn_noalloc.cu"),
+           "-o", lib]
     res = subprocess.run(cmd, capture_output=True, text=True)
     if res.returncode != 0:
         sys.stderr.write(res.stdout + res.stderr)
         raise RuntimeError("nvcc failed building the attention library")
     if verbose:
         sys.stderr.write(res.stderr)
-    check_register_budget(res.stdout + res.stderr)
-    return LIB
+    check_register_budget(res.stdout + res.stderr, lib)
+    return lib
 
 
 # The prefill kernel redistributes registers with setmaxnreg assuming each of
@@ -64,7 +69,7 @@ FWD_LAUNCH_REGS = 168
 BWD_LAUNCH_REGS = 96
 
 
-def check_register_budget(ptxas_log: str) -> None:
+def check_register_budget(ptxas_log: str, lib: str = LIB) -> None:
     current = None
     seen = 0
     seen_bwd = 0
@@ -77,19 +82,19 @@ def check_register_budget(ptxas_log: str) -> None:
         if m and current and "attn_bwd_sm100_kernel" in current:
             seen_bwd += 1
             if int(m.group(1)) != BWD_LAUNCH_REGS:
-                os.remove(LIB)
+                os.remove(lib)
                 raise RuntimeError(f"{current} uses {m.group(1)} registers, expected "
                                    f"{BWD_LAUNCH_REGS}: the setmaxnreg split would not fit")
         if m and current and "attn_fwd_sm100_kernel" in current:
             seen += 1
             if int(m.group(1)) != FWD_LAUNCH_REGS:
-                os.remove(LIB)
+                os.remove(lib)
                 raise RuntimeError(f"{current} uses {m.group(1)} registers, expected "
                                    f"{FWD_LAUNCH_REGS}: the setmaxnreg split would not fit")
     if seen == 0 or seen_bwd == 0:
-        os.remove(LIB)
+        os.remove(lib)
         raise RuntimeError("ptxas register report for the prefill or backward kernel not found")
 
 
 if __name__ == "__main__":
-    print(build(force="--force" in sys.argv, verbose=True))
+    print(build(force="--force" in sys.argv, verbose=True, debug="--debug" in sys.argv))

@@ -12,6 +12,7 @@
 #include <atomic>
 #include <cmath>
 #include <cstdint>
+#include <cstdlib>
 #include <cstring>
 #include <mutex>
 
@@ -136,6 +137,13 @@ int fwd_group_heads(int BH, int Nkv, int d, int elem_bytes) {
     if (g < 1) g = 1;
     return g < BH ? (int)g : BH;
 }
+// Units are dealt dynamically, in head groups, only when the K and V of all
+// heads exceed this (the launch's K/V then cannot stay in the 126 MB L2 while
+// every head is in flight); below it a static deal of the heaviest-first
+// order is used. 0 forces the dynamic queue, a huge value the static deal.
+#ifndef EATTN_FWD_QUEUE_MIN_BYTES
+#define EATTN_FWD_QUEUE_MIN_BYTES (192ll << 20)
+#endif
 
 template <int D, bool CAUSAL, bool FP8 = false>
 attn_status_t launch_fwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
@@ -161,7 +169,15 @@ attn_status_t launch_fwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUt
         sms = di.sms;
     }
     const int grid = p.num_units < sms ? p.num_units : sms;
-    p.group_heads = fwd_group_heads(p.BH, p.Nkv, D, T::kElemBytes);
+    p.dynamic_units =
+        2ll * p.BH * p.Nkv * D * T::kElemBytes > EATTN_FWD_QUEUE_MIN_BYTES ? 1 : 0;
+    // EXACT_ATTN_FWD_SCHEDULE=dynamic|static overrides the choice (for tests
+    // and measurements; the result is the same either way)
+    if (const char* sched = std::getenv("EXACT_ATTN_FWD_SCHEDULE")) {
+        if (std::strcmp(sched, "dynamic") == 0) p.dynamic_units = 1;
+        if (std::strcmp(sched, "static") == 0) p.dynamic_units = 0;
+    }
+    p.group_heads = p.dynamic_units ? fwd_group_heads(p.BH, p.Nkv, D, T::kElemBytes) : p.BH;
     p.queue_slot = (int)(g_fwd_queue_rr.fetch_add(1, std::memory_order_relaxed) % kFwdQueueSlots);
     kern<<<grid, T::kThreads, T::kSmemBytes, stream>>>(tq, tk, tv, p);
     return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
@@ -224,6 +240,8 @@ const char* attn_strerror(attn_status_t s) {
             return "partials exceed the library's fixed 32 MiB decode scratch array";
         case ATTN_ERR_BAD_INDEX:
             return "a block-table entry or sequence length was out of range; those keys were skipped";
+        case ATTN_ERR_INDEX_CHECK:
+            return "debug build: a kernel computed an index outside its tensor; the access was skipped";
     }
     return "unknown status";
 }
@@ -572,6 +590,7 @@ attn_status_t attn_status(void* stream) {
     }
     if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
     if (word & kDevErrTimeout) return ATTN_ERR_TIMEOUT;
+    if (word & kDevErrIndexCheck) return ATTN_ERR_INDEX_CHECK;
     if (word & kDevErrBadIndex) return ATTN_ERR_BAD_INDEX;
     return ATTN_OK;
 }

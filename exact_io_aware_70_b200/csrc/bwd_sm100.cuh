@@ -62,7 +62,7 @@ __global__ void __launch_bounds__(256) attn_bwd_preprocess_kernel(const BwdParam
     const bool in_range = row < (long long)p.BH * p.NqPad;
     const long long bh = in_range ? row / p.NqPad : 0;
     const int i = in_range ? (int)(row % p.NqPad) : 0;
-    const bool real = in_range && i < p.Nq;
+    const bool real = in_range && i < p.Nq && dcheck(bh < p.BH);
     const long long grow = bh * p.Nq + i;
     float acc = 0.f;
     if (real) {
@@ -375,10 +375,10 @@ __global__ void __launch_bounds__(640, 1)
             if (quarter * 32 < D) {
                 float* dq_rows = dq_head + (size_t)row0 * D;
                 const int nr = p.Nq - row0;   // rows of this block inside the head
-                if (nr >= 32) {
+                if (nr >= 32 && dcheck(row0 + 32 <= p.Nq && bh < p.BH)) {
 #pragma unroll
                     for (int e = 0; e < 32; ++e) red_add_f32(dq_rows + e * D, __uint_as_float(v[e]));
-                } else {
+                } else if (nr < 32) {
 #pragma unroll
                     for (int e = 0; e < 32; ++e)
                         if (e < nr) red_add_f32(dq_rows + e * D, __uint_as_float(v[e]));

@@ -190,6 +190,7 @@ __global__ void __launch_bounds__(256, PAGED ? 4 : 1)
     const long long j1 = min(j0 + (long long)L, (long long)nkv);
     const int n = j1 > j0 ? (int)(j1 - j0) : 0;
     float* o_out = p.o_part + ((size_t)bh * p.S + c) * D;
+    if (!dcheck(c < p.S && (!PAGED || b < (int)gridDim.y / p.H))) return;
 
     if (n == 0) {   // empty chunk: weight zero in the merge
         for (int x = tid; x < D; x += blockDim.x) o_out[x] = 0.f;
@@ -253,8 +254,9 @@ __global__ void __launch_bounds__(256, PAGED ? 4 : 1)
                     kr[r] = page >= 0 ? ld_stream_16B(kpaged + paged_offset(sb + i, page), pol)
                                       : make_uint4(0, 0, 0, 0);
                 } else {
-                    kr[r] = i < nsub ? ld_stream_16B(kbase + (size_t)(sb + i) * D, pol)
-                                     : make_uint4(0, 0, 0, 0);
+                    kr[r] = (i < nsub && dcheck(j0 + sb + i < p.Nkv))
+                                ? ld_stream_16B(kbase + (size_t)(sb + i) * D, pol)
+                                : make_uint4(0, 0, 0, 0);
                 }
             }
             float part[8];
@@ -317,8 +319,9 @@ __global__ void __launch_bounds__(256, PAGED ? 4 : 1)
                     vr[r] = page >= 0 ? ld_stream_16B(vpaged + paged_offset(sb + i, page), pol)
                                       : make_uint4(0, 0, 0, 0);
                 } else {
-                    vr[r] = i < nsub ? ld_stream_16B(vbase + (size_t)(sb + i) * D, pol)
-                                     : make_uint4(0, 0, 0, 0);
+                    vr[r] = (i < nsub && dcheck(j0 + sb + i < p.Nkv))
+                                ? ld_stream_16B(vbase + (size_t)(sb + i) * D, pol)
+                                : make_uint4(0, 0, 0, 0);
                 }
             }
 #pragma unroll
@@ -379,7 +382,8 @@ __global__ void __launch_bounds__(kMergeThreads)
     // chunk c (0 <= c < C) of this row: group c / S, chunk c % S within it
     auto row_of = [&](int c) -> size_t {
         const int r = c / S;
-        return ((size_t)r * BH + bh) * S + (c - r * S);
+        const size_t row = ((size_t)r * BH + bh) * S + (c - r * S);
+        return dcheck(row < (size_t)R * BH * S) ? row : 0;
     };
     // ---- M = max_c lse_c
     float M = -INFINITY;

@@ -14,10 +14,11 @@
 // How it maps onto a B200 SM (this design is ours; the pages' A100/H100
 // kernels are prior art only):
 //   * Persistent grid, one CTA per SM. A work unit is (batch*head, 256 query
-//     rows) = two 128-row Q tiles. Units are sorted heaviest-first and dealt
-//     to the CTAs in alternating direction each round (CTA i takes unit
-//     r*G + i in even rounds, r*G + G-1-i in odd rounds), which balances the
-//     causal triangle across the 148 SMs about as well as longest-first greedy.
+//     rows) = two 128-row Q tiles. CTAs take units from a device counter as
+//     they become free (a dynamic queue), in an order that groups the heads so
+//     that the K/V of the heads in flight stays in L2 and that goes
+//     heaviest-first inside a group (longest-first balance of the causal
+//     triangle); see fwd_fetch_unit.
 //   * Warp 8 is the TMA producer (lane 0 issues): Q tiles once per unit,
 //     then K_j and V_j tiles into a ring of shared-memory slots, 128-byte
 //     swizzled, completion counted on mbarriers.
@@ -55,8 +56,14 @@
 //     that costs the MMA issuer one more barrier check per tile and step and
 //     measured slower). K_j and V_j complete on one barrier, and each Q tile is
 //     released to the producer right after its last S product of the unit.
-//   * Tensor memory columns: S0 [0,128), S1 [128,256), O0 [256,256+d),
-//     O1 [256+d, 256+2d).
+//   * Tensor memory columns, head dim 128: S0 [0,128), S1 [128,256), O0
+//     [256,384), O1 [384,512); S_t(j+1) overwrites P_t(j), so it is issued
+//     after P_t(j) V. Head dim 64: three score buffers [0,384) used in
+//     rotation, O0 [384,448), O1 [448,512); S_t(j+1) is computed one step
+//     ahead, while the softmax group still works on S_t(j) (fwd_mma_ahead).
+//   * Epilogue: O / l in bf16 goes through a 2 KB shared-memory block per
+//     warp so that each global store instruction writes whole rows' 64-byte
+//     pieces (full 32-byte sectors) rather than one 16-byte piece of 32 rows.
 //   * The same kernel serves e4m3 inputs (FP8 = true): tiles of one swizzle
 //     panel (16 KB of 128-byte rows at d=128, an 8-slot K/V ring; 8 KB of
 //     64-byte rows with the 64-byte swizzle at d=64, 16 slots), both products as
@@ -87,6 +94,7 @@ struct FwdParams {
     int num_qb;         // ceil(Nq / 256)
     int num_units;      // BH * num_qb
     int group_heads;    // heads per group of the unit order (see fwd_unit)
+    int dynamic_units;  // 1: units come from the device counter; 0: static snake deal
     int queue_slot;     // which entry of g_fwd_queues this launch counts its units in
     float scale_log2;   // scale * log2(e)
 };
@@ -107,6 +115,17 @@ struct FwdParams {
 // 1: P is released to the MMA issuer in two halves (p_lo, p_hi); 0: once.
 #ifndef EATTN_SPLIT_P
 #define EATTN_SPLIT_P 0
+#endif
+
+// 1: at head dim 64 the score products rotate over three TMEM buffers and run
+//    one step ahead of the softmax (fwd_mma_ahead); 0: two fixed buffers.
+#ifndef EATTN_SBUFS_AHEAD
+#define EATTN_SBUFS_AHEAD 1
+#endif
+// 1: the epilogue's O stores go through shared memory as row-contiguous
+//    64-byte pieces (full sectors); 0: each thread stores its own row.
+#ifndef EATTN_STAGE_O
+#define EATTN_STAGE_O 1
 #endif
 
 // FP8 = true: Q, K, V are e4m3 codes with per-(batch*head) descale factors;
@@ -165,7 +184,7 @@ struct FwdTraits {
     // With three (head dim 64: 3 x 128 + 2 x 64 = 512) the S products rotate
     // over the buffers in issue order and S_t(j+1) is computed ahead, while
     // the softmax still works on S_t(j) (see fwd_mma).
-    static constexpr int kSBufs = (3 * 128 + 2 * D <= 512) ? 3 : 2;
+    static constexpr int kSBufs = (EATTN_SBUFS_AHEAD && 3 * 128 + 2 * D <= 512) ? 3 : 2;
     static constexpr uint32_t kColS0 = 0, kColS1 = 128;
     static constexpr uint32_t kColO0 = 128 * kSBufs, kColO1 = 128 * kSBufs + D;
 };
@@ -205,9 +224,22 @@ constexpr int kPolyEvery =
 constexpr int kFwdQueueSlots = 64;
 __device__ int g_fwd_queues[2 * kFwdQueueSlots];
 
-__device__ __forceinline__ int fwd_fetch_unit(const FwdParams& p) {
-    const int u = atomicAdd(&g_fwd_queues[2 * p.queue_slot], 1);
-    return u < p.num_units ? u : -1;
+// The unit a CTA's producer publishes as its round-th unit. Dynamic: the next
+// index of the device counter. Static (used when the K/V of all heads fit in
+// L2, where grouping gains nothing and the counter's latency would only
+// delay each unit): a snake deal of the same order -- CTA i takes index
+// r * G + i in even rounds and r * G + G - 1 - i in odd ones (G = grid size),
+// which balances the heaviest-first order about as well as longest-first
+// greedy.
+__device__ __forceinline__ int fwd_fetch_unit(const FwdParams& p, uint32_t round) {
+    long long u;
+    if (p.dynamic_units) {
+        u = atomicAdd(&g_fwd_queues[2 * p.queue_slot], 1);
+    } else {
+        const int g = gridDim.x, i = blockIdx.x;
+        u = (long long)round * g + ((round & 1) ? (g - 1 - i) : i);
+    }
+    return u < p.num_units ? (int)u : -1;
 }
 
 struct FwdUnit {
@@ -225,6 +257,7 @@ __device__ __forceinline__ FwdUnit fwd_unit(int u, const FwdParams& p) {
     const int heads = min(p.group_heads, p.BH - g * p.group_heads);   // the last group may be short
     x.qb = p.num_qb - 1 - r / heads;   // heaviest (latest) query blocks first
     x.bh = g * p.group_heads + r % heads;
+    dcheck(x.qb >= 0 && x.bh < p.BH);
 #pragma unroll
     for (int t = 0; t < 2; ++t) {
         const long long r0 = (long long)x.qb * 256 + t * 128;
@@ -341,7 +374,7 @@ __device__ void fwd_producer(const FwdParams& p, const CUtensorMap* tq, const CU
     const uint64_t pol_kv = l2_policy_evict_last();
     uint32_t kv_iter = 0;
     uint32_t q_issued[2] = {0, 0};
-    int u = fwd_fetch_unit(p);
+    int u = fwd_fetch_unit(p, 0);
     for (uint32_t k = 0;; ++k) {
         // publish unit u (or the end) in ring entry k once its last readers are done
         const int slot = k & 1;
@@ -365,7 +398,7 @@ __device__ void fwd_producer(const FwdParams& p, const CUtensorMap* tq, const CU
                                   pn * T::kPanelElems, x.qb * 256 + t * 128, x.bh, leader);
             ++q_issued[t];
         }
-        u = fwd_fetch_unit(p);   // the next unit, fetched while this one's tiles stream in
+        u = fwd_fetch_unit(p, k + 1);   // the next unit, fetched while this one's tiles stream in
         for (int j = 0; j < x.nmax; ++j) {
 #pragma unroll
             for (int which = 0; which < 2; ++which) {   // K_j, then V_j
@@ -682,7 +715,8 @@ __device__ __forceinline__ uint32_t stage_slot(int r, int k) {
 
 template <int D>
 __device__ __forceinline__ void fwd_store_chunk(uint32_t stage, const uint32_t (&w)[16], int lane,
-                                                uint16_t* o_rows, int c, int valid_rows) {
+                                                uint16_t* o_rows, int c, int valid_rows,
+                                                const uint16_t* o_end) {
     __syncwarp();   // the previous chunk's reads of the staging block are done
 #pragma unroll
     for (int k = 0; k < 4; ++k)
@@ -693,8 +727,8 @@ __device__ __forceinline__ void fwd_store_chunk(uint32_t stage, const uint32_t (
     for (int i = 0; i < 4; ++i) {
         const int r = i * 8 + (lane >> 2), k = lane & 3;
         const uint4 val = ld_shared_v4(stage + stage_slot(r, k));
-        if (r < valid_rows)
-            *reinterpret_cast<uint4*>(o_rows + (size_t)r * D + c + 8 * k) = val;
+        uint16_t* dst = o_rows + (size_t)r * D + c + 8 * k;
+        if (r < valid_rows && dcheck(dst + 8 <= o_end)) *reinterpret_cast<uint4*>(dst) = val;
     }
 }
 
@@ -873,17 +907,25 @@ __device__ void fwd_softmax(const FwdParams& p, uint32_t tbase,
                 for (int i = 0; i < 16; ++i)
                     w[i] = pack_bf16x2(__uint_as_float(orr[2 * i]) * inv,
                                        __uint_as_float(orr[2 * i + 1]) * inv);
-                fwd_store_chunk<D>(stage, w, lane, o_rows, c, valid_rows);
+                if (EATTN_STAGE_O) {
+                    fwd_store_chunk<D>(stage, w, lane, o_rows, c, valid_rows,
+                                       p.o + (size_t)p.BH * p.Nq * D);
+                } else if (row_valid && dcheck(x.bh < p.BH)) {
+                    uint4* dst = reinterpret_cast<uint4*>(orow + c);
+#pragma unroll
+                    for (int k4 = 0; k4 < 4; ++k4)
+                        dst[k4] = make_uint4(w[4 * k4], w[4 * k4 + 1], w[4 * k4 + 2], w[4 * k4 + 3]);
+                }
             }
             tc_fence_before_sync();
             mbar_arrive(bar_ofree);
             ++o_use;
-        } else if (row_valid) {
+        } else if (row_valid && dcheck(x.bh < p.BH)) {
             uint4* dst = reinterpret_cast<uint4*>(orow);
 #pragma unroll
             for (int k = 0; k < D / 8; ++k) dst[k] = make_uint4(0, 0, 0, 0);
         }
-        if (row_valid)
+        if (row_valid && dcheck(x.bh < p.BH))
             p.lse[(size_t)x.bh * p.Nq + qrow] =
                 l > 0.f ? (m_ref - T::kShift + log2f(l)) * 0.69314718055994531f : -INFINITY;
     }
@@ -977,7 +1019,7 @@ __global__ void __launch_bounds__(384, 1)
     }
     // Every role of this CTA is done, so its producer has made its last fetch.
     // The CTA that finishes last returns the queue to zero for the next launch.
-    if (threadIdx.x == 0) {
+    if (threadIdx.x == 0 && p.dynamic_units) {
         int* q = &g_fwd_queues[2 * p.queue_slot];
         __threadfence();
         if (atomicAdd(q + 1, 1) == (int)gridDim.x - 1) {

@@ -16,6 +16,26 @@ namespace eattn {
 
 // Bits of the device status word (read and cleared by attn_status()).
 constexpr unsigned kDevErrTimeout = 1u;
+// (bit 2u, kDevErrBadIndex, belongs to the paged decode)
+constexpr unsigned kDevErrIndexCheck = 4u;
+
+// Index checks of the debug build (compiled with -DATTN_DEBUG). The kernels
+// guard their global-memory accesses that use computed indices with
+// `if (dcheck(index < limit))`: in the debug build a failed check records
+// kDevErrIndexCheck in the device status word (attn_status() then reports
+// ATTN_ERR_INDEX_CHECK) and the access is skipped, so a wrong index shows up
+// as an error instead of a stray write; nothing traps. In the normal build
+// dcheck is the constant true and the checks compile away. (g_attn_status is
+// defined by the translation unit that includes the kernels, before them.)
+__device__ __forceinline__ bool dcheck(bool ok) {
+#ifdef ATTN_DEBUG
+    if (!ok) atomicOr(&g_attn_status, kDevErrIndexCheck);
+    return ok;
+#else
+    (void)ok;
+    return true;
+#endif
+}
 
 // Wall-time limit of one pipeline wait. Real waits last microseconds.
 constexpr unsigned long long kWaitLimitNs = 1000ull * 1000ull * 1000ull;  // 1 s

@@ -51,7 +51,8 @@ typedef enum {
     ATTN_ERR_CUDA = 4,
     ATTN_ERR_TIMEOUT = 5,
     ATTN_ERR_SCRATCH_LIMIT = 6,
-    ATTN_ERR_BAD_INDEX = 7
+    ATTN_ERR_BAD_INDEX = 7,
+    ATTN_ERR_INDEX_CHECK = 8
 } attn_status_t;
 
 /* Version of this ABI (bumped on any incompatible change). */
@@ -300,6 +301,9 @@ attn_status_t attn_bwd(const void *q, const void *k, const void *v, const void *
  * ATTN_ERR_TIMEOUT if a kernel's pipeline wait gave up since the last call
  * (its outputs are then invalid), ATTN_ERR_BAD_INDEX if a paged decode met an
  * out-of-range block-table entry or length (those keys were skipped),
+ * ATTN_ERR_INDEX_CHECK if, in the debug build of the library (compiled with
+ * -DATTN_DEBUG), a kernel computed a global-memory index outside its tensor
+ * (the access was skipped; the normal build does not check),
  * ATTN_ERR_CUDA if the stream reported an error, ATTN_OK otherwise.
  */
 attn_status_t attn_status(void *stream);

@@ -48,7 +48,7 @@ def test_library_exports_every_declared_symbol(ea):
 
 def test_version_and_strerror(ea):
     assert ea.abi_version() == 1
-    for code in range(6):
+    for code in range(9):
         assert ea.attn_strerror(code)
     assert "unknown" in ea.attn_strerror(99)
 
@@ -186,3 +186,19 @@ def test_package_fails_loudly_without_the_library(tmp_path):
     with pytest.raises(ImportError, match="missing"):
         spec.loader.exec_module(mod)
     sys.modules.pop("fake_pkg", None)
+
+
+def test_debug_build_compiles_and_exports_every_symbol():
+    """The index-checking debug build (-DATTN_DEBUG) of the same sources builds
+    for sm_100a and exports the same entry points."""
+    spec = importlib.util.spec_from_file_location(
+        "exact_attn_cuda_build", os.path.join(ROOT, "exact_io_aware_70_b200", "build.py"))
+    build = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(build)
+    path = build.build(debug=True)
+    assert path.endswith("libexact_attn_b200_debug.so")
+    lib = ctypes.CDLL(path)
+    for name in declared_functions():
+        assert hasattr(lib, name), f"{name} missing from the debug build"
+    lib.attn_strerror.restype = ctypes.c_char_p
+    assert b"debug build" in lib.attn_strerror(8)

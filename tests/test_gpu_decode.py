@@ -6,7 +6,7 @@ import torch
 import oracle
 from seeded_inputs import WORKLOADS, bf16_bits, make_partials, make_qkv, make_workload
 from tests import gpu_util
-from tests.parity import LSE_MAX_ABS, compare
+from tests.parity import LSE_MAX_ABS, compare, compare_merge
 
 pytestmark = pytest.mark.gpu
 
@@ -77,7 +77,7 @@ def test_lse_merge_matches_oracle(d, S, empty_every):
     m.attn_lse_merge(o_p.cuda(), l_p.cuda(), o, lse)
     assert m.attn_status() == 0
     ro, rl = oracle.get().lse_merge_f32in(o_p.numpy(), l_p.numpy())
-    compare(o[:, :, 0].float().cpu().numpy(), lse[:, :, 0].cpu().numpy(), ro, rl, "merge")
+    compare_merge(o[:, :, 0].float().cpu().numpy(), lse[:, :, 0].cpu().numpy(), ro, rl, "merge")
 
 
 def test_decode_deterministic():

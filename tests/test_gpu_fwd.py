@@ -71,6 +71,23 @@ def test_fwd_sweep(shape):
     gpu_util.fwd_full_parity(B, H, Nq, Nkv, d, causal, seed=100 + Nq + Nkv + d)
 
 
+@pytest.fixture
+def schedule(monkeypatch, request):
+    """Force the forward's unit deal (the library reads EXACT_ATTN_FWD_SCHEDULE
+    on every call): the dynamic queue normally serves only launches whose K/V
+    exceed L2, the static deal the rest."""
+    monkeypatch.setenv("EXACT_ATTN_FWD_SCHEDULE", request.param)
+    return request.param
+
+
+@pytest.mark.parametrize("schedule", ["dynamic", "static"], indirect=True)
+@pytest.mark.parametrize("shape", [SWEEP[i] for i in (1, 6, 9, 16, 18, 19, 20, 21)],
+                         ids=lambda s: "B{}H{}q{}kv{}d{}c{}".format(*s[:5], int(s[5])))
+def test_fwd_sweep_both_schedules(shape, schedule):
+    B, H, Nq, Nkv, d, causal = shape
+    gpu_util.fwd_full_parity(B, H, Nq, Nkv, d, causal, seed=100 + Nq + Nkv + d)
+
+
 def test_tiny_workload():
     w = WORKLOADS["tiny"]
     gpu_util.fwd_full_parity(w.B, w.H, w.Nq, w.Nkv, w.d, w.causal, w.seed, scale=w.scale)
@@ -128,7 +145,8 @@ def test_deterministic():
     assert torch.equal(o1, o2) and torch.equal(l1, l2)
 
 
-def test_concurrent_launches_on_two_streams():
+@pytest.mark.parametrize("schedule", ["dynamic"], indirect=True)
+def test_concurrent_launches_on_two_streams(schedule):
     """Launches in flight at the same time on two streams take their work units
     from different queue entries, so neither steals the other's units."""
     from seeded_inputs import make_qkv

@@ -16,7 +16,7 @@ import oracle
 from exact_io_aware_70_b200.sharding import kv_range
 from seeded_inputs import bf16_bits, make_partials, make_qkv
 from tests import gpu_util
-from tests.parity import compare
+from tests.parity import compare, compare_merge
 
 pytestmark = pytest.mark.gpu
 
@@ -62,7 +62,8 @@ def test_gathered_merge_matches_oracle_merge(R, S, d, empty_every):
     m.attn_lse_merge_gathered(og.cuda(), lg.cuda(), o, lse)
     assert m.attn_status() == 0
     ro, rl = oracle.get().lse_merge_f32in(o_p.numpy(), l_p.numpy())
-    compare(o[:, :, 0].float().cpu().numpy(), lse[:, :, 0].cpu().numpy(), ro, rl, "gathered merge")
+    compare_merge(o[:, :, 0].float().cpu().numpy(), lse[:, :, 0].cpu().numpy(), ro, rl,
+                  "gathered merge")
 
 
 def test_merge_reads_unaligned_partials():
@@ -81,5 +82,6 @@ def test_merge_reads_unaligned_partials():
     m.attn_lse_merge(op, l_p.cuda(), o, lse)
     assert m.attn_status() == 0
     ro, rl = oracle.get().lse_merge_f32in(o_p.numpy(), l_p.numpy())
-    compare(o[:, :, 0].float().cpu().numpy(), lse[:, :, 0].cpu().numpy(), ro, rl, "unaligned merge")
+    compare_merge(o[:, :, 0].float().cpu().numpy(), lse[:, :, 0].cpu().numpy(), ro, rl,
+                  "unaligned merge")
     assert obuf[0].item() == 0.0

@@ -122,6 +122,10 @@ struct FwdParams {
 #ifndef EATTN_SBUFS_AHEAD
 #define EATTN_SBUFS_AHEAD 1
 #endif
+// 1: two sets of Q tiles where shared memory allows (see FwdTraits::kQBufs)
+#ifndef EATTN_Q_DOUBLE
+#define EATTN_Q_DOUBLE 1
+#endif
 // 1: the epilogue's O stores go through shared memory as row-contiguous
 //    64-byte pieces (full sectors); 0: each thread stores its own row.
 #ifndef EATTN_STAGE_O
@@ -170,12 +174,18 @@ struct FwdTraits {
     static constexpr int kOtherRegs = 120;
     static_assert(2 * 128 * kSoftmaxRegs + 128 * kOtherRegs <= kThreads * kLaunchRegs,
                   "register split exceeds the launch allocation");
-    static constexpr int kNumBars = 2 * kSlots + 23;   // FwdBars<kSlots>::kCount
+    static constexpr int kNumBars = 2 * kSlots + 27;   // FwdBars<kSlots>::kCount
     // epilogue staging: one 32-row x 64-byte (32 bf16 columns) block per softmax warp
     static constexpr int kStageWarpBytes = 32 * 64;
     static constexpr int kStageBytes = 8 * kStageWarpBytes;
+    // Q tiles: two (one unit's), or four where shared memory allows (head dim
+    // 64, and e4m3 inputs), so that the next unit's Q is loaded while this
+    // unit still runs instead of after its last S product
+    static constexpr int kQBufs =
+        (EATTN_Q_DOUBLE &&
+         1024 + (4 + kSlots) * kTileBytes + kStageBytes + kNumBars * 8 + 32 <= 232448) ? 4 : 2;
     static constexpr int kSmemBytes =
-        1024 + (2 + kSlots) * kTileBytes + kStageBytes + kNumBars * 8 + 16 + 16;
+        1024 + (kQBufs + kSlots) * kTileBytes + kStageBytes + kNumBars * 8 + 16 + 16;
     static_assert(kSmemBytes <= 232448, "shared memory per CTA");
     static constexpr uint32_t kTmemCols = 512;
     // Score buffers of 128 fp32 columns. With two (head dim 128: 2 x 128 + 2 x
@@ -287,14 +297,19 @@ __device__ __forceinline__ int fwd_s_pos(const FwdUnit& x, int t, int i) {
 // only a single register is live across the roles. Layout (8 bytes each):
 // kv_full[S], kv_empty[S], then 2 each of q_full, q_empty, s_full, p_lo, p_hi,
 // o_final, o_free, then drain, then 2 each of unit_full, unit_empty, s_full_b,
-// pv_done.
+// pv_done, and of q_full, q_empty for the second set of Q tiles.
 template <int S>
 struct FwdBars {
     uint32_t base;
     __device__ __forceinline__ uint32_t kv_full(uint32_t i) const { return base + 8 * i; }
     __device__ __forceinline__ uint32_t kv_empty(uint32_t i) const { return base + 8 * (S + i); }
-    __device__ __forceinline__ uint32_t q_full(int t) const { return base + 8 * (2 * S + t); }
-    __device__ __forceinline__ uint32_t q_empty(int t) const { return base + 8 * (2 * S + 2 + t); }
+    // Q tile slot qi = 2 * set + t (set 1 exists only with four Q tiles)
+    __device__ __forceinline__ uint32_t q_full(int qi) const {
+        return base + 8 * (qi < 2 ? 2 * S + qi : 2 * S + 23 + (qi - 2));
+    }
+    __device__ __forceinline__ uint32_t q_empty(int qi) const {
+        return base + 8 * (qi < 2 ? 2 * S + 2 + qi : 2 * S + 25 + (qi - 2));
+    }
     __device__ __forceinline__ uint32_t s_full(int t) const { return base + 8 * (2 * S + 4 + t); }
     __device__ __forceinline__ uint32_t p_lo(int t) const { return base + 8 * (2 * S + 6 + t); }
     __device__ __forceinline__ uint32_t p_hi(int t) const { return base + 8 * (2 * S + 8 + t); }
@@ -317,7 +332,7 @@ struct FwdBars {
     static __device__ __forceinline__ uint32_t s_parity(uint32_t c) {
         return kSBufs == 3 ? (c >> 1) & 1 : c & 1;
     }
-    static constexpr int kCount = 2 * S + 23;
+    static constexpr int kCount = 2 * S + 27;
     // shared-memory words after the barriers: TMEM base, abort flag, unit ring[2]
     __device__ __forceinline__ volatile int* unit_slot(int i) const {
         return reinterpret_cast<volatile int*>(unit_ring_ptr) + i;
@@ -329,12 +344,18 @@ struct FwdBars {
 // softmax warps.
 constexpr int kUnitReaders = 9;
 
-// Next unit for a consumer role: waits for ring entry k, reads it and
-// releases the entry (the MMA issuer and lane 0 of each softmax warp count as
-// its readers). Returns false on a failed wait; *u = -1 marks the end.
+// Next unit for a consumer role. Dynamic deal: waits for ring entry k, reads
+// it and releases the entry (the MMA issuer and lane 0 of each softmax warp
+// count as its readers). Static deal: the k-th unit of the snake deal. Returns
+// false on a failed wait; *u = -1 marks the end.
 template <int S>
-__device__ __forceinline__ bool fwd_next_unit(const FwdBars<S>& b, uint32_t k, bool arrive,
-                                              volatile int* abort_flag, int* u) {
+__device__ __forceinline__ bool fwd_next_unit(const FwdParams& p, const FwdBars<S>& b, uint32_t k,
+                                              bool arrive, volatile int* abort_flag, int* u) {
+    // the static deal needs no hand-over: every role computes the same sequence
+    if (!p.dynamic_units) {
+        *u = fwd_fetch_unit(p, k);
+        return true;
+    }
     const int slot = k & 1;
     if (!mbar_wait(b.unit_full(slot), (k >> 1) & 1, abort_flag, &g_attn_status)) return false;
     *u = *b.unit_slot(slot);
@@ -373,30 +394,38 @@ __device__ void fwd_producer(const FwdParams& p, const CUtensorMap* tq, const CU
     const uint64_t pol_q = l2_policy_evict_first();
     const uint64_t pol_kv = l2_policy_evict_last();
     uint32_t kv_iter = 0;
-    uint32_t q_issued[2] = {0, 0};
+    uint32_t q_issued[4] = {0, 0, 0, 0};
     int u = fwd_fetch_unit(p, 0);
     for (uint32_t k = 0;; ++k) {
-        // publish unit u (or the end) in ring entry k once its last readers are done
-        const int slot = k & 1;
-        if (k >= 2 && !role_wait(b.unit_empty(slot), ((k >> 1) - 1) & 1, abort_flag)) goto fail;
-        *b.unit_slot(slot) = u;
-        mbar_arrive(b.unit_full(slot));
+        // dynamic deal: publish unit u (or the end) in ring entry k once its last
+        // readers are done (the static deal needs no hand-over)
+        if (p.dynamic_units) {
+            const int slot = k & 1;
+            if (k >= 2 && !role_wait(b.unit_empty(slot), ((k >> 1) - 1) & 1, abort_flag))
+                goto fail;
+            *b.unit_slot(slot) = u;
+            mbar_arrive(b.unit_full(slot));
+        }
         if (u < 0) break;
         const FwdUnit x = fwd_unit<CAUSAL>(u, p);
+        const int qset = T::kQBufs == 4 ? (int)(k & 1) : 0;
         for (int t = 0; t < 2; ++t) {
-            if (q_issued[t] > 0 && !role_wait(b.q_empty(t), (q_issued[t] - 1) & 1, abort_flag))
+            const int qi = 2 * qset + t;
+            if (q_issued[qi] > 0 &&
+                !role_wait(b.q_empty(qi), (q_issued[qi] - 1) & 1, abort_flag))
                 goto fail;
-            mbar_arrive_expect_tx_w(b.q_full(t), T::kTileBytes, leader);
+            mbar_arrive_expect_tx_w(b.q_full(qi), T::kTileBytes, leader);
 #pragma unroll
             for (int pn = 0; pn < T::kPanels; ++pn)
                 if (EATTN_FWD_L2_HINTS)
-                    tma_load_3d_hint_w(sQ + t * T::kTileBytes + pn * T::kPanelBytes, tq,
-                                       b.q_full(t), pn * T::kPanelElems, x.qb * 256 + t * 128,
+                    tma_load_3d_hint_w(sQ + qi * T::kTileBytes + pn * T::kPanelBytes, tq,
+                                       b.q_full(qi), pn * T::kPanelElems, x.qb * 256 + t * 128,
                                        x.bh, pol_q, leader);
                 else
-                    tma_load_3d_w(sQ + t * T::kTileBytes + pn * T::kPanelBytes, tq, b.q_full(t),
-                                  pn * T::kPanelElems, x.qb * 256 + t * 128, x.bh, leader);
-            ++q_issued[t];
+                    tma_load_3d_w(sQ + qi * T::kTileBytes + pn * T::kPanelBytes, tq,
+                                  b.q_full(qi), pn * T::kPanelElems, x.qb * 256 + t * 128, x.bh,
+                                  leader);
+            ++q_issued[qi];
         }
         u = fwd_fetch_unit(p, k + 1);   // the next unit, fetched while this one's tiles stream in
         for (int j = 0; j < x.nmax; ++j) {
@@ -436,9 +465,9 @@ fail: {
     for (uint32_t i = first; i < kv_iter; ++i)
         if (!EATTN_KV_PAIR_BARRIER || (i % 2) == 0)
             mbar_wait(b.kv_full(i % T::kSlots), (i / T::kSlots) & 1, &no_abort, &g_attn_status);
-    for (int t = 0; t < 2; ++t)
-        if (q_issued[t] > 0)
-            mbar_wait(b.q_full(t), (q_issued[t] - 1) & 1, &no_abort, &g_attn_status);
+    for (int qi = 0; qi < T::kQBufs; ++qi)
+        if (q_issued[qi] > 0)
+            mbar_wait(b.q_full(qi), (q_issued[qi] - 1) & 1, &no_abort, &g_attn_status);
 }
 }
 
@@ -514,25 +543,27 @@ __device__ void fwd_mma_ahead(const FwdParams& p, uint32_t tbase, uint32_t sQ, u
     const uint64_t dk0 = fwd_sdesc<T>(sKV, 16);                       // K-major K tile
     const uint64_t dv0 = fwd_sdesc<T>(sKV, T::kPanelBytes);           // MN-major V tile
     const uint32_t colO[2] = {T::kColO0, T::kColO1};
-    uint32_t kv_iter = 0, q_use = 0, s_issued = 0;
+    uint32_t kv_iter = 0, s_issued = 0;
+    uint32_t q_use[2] = {0, 0};     // units that used Q set 0 / set 1
     uint32_t o_use[2] = {0, 0}, p_cnt[2] = {0, 0}, s_cnt[2] = {0, 0};
     uint32_t cur_col[2] = {0, 0};   // buffer holding S_t(j) / P_t(j)
     for (uint32_t k = 0;; ++k) {
         int u;
-        if (!fwd_next_unit(b, k, true, abort_flag, &u)) goto done;
+        if (!fwd_next_unit(p, b, k, true, abort_flag, &u)) goto done;
         if (u < 0) break;
         {
             const FwdUnit x = fwd_unit<CAUSAL>(u, p);
-            if (!role_wait(b.q_full(0), q_use & 1, abort_flag)) goto done;
-            if (!role_wait(b.q_full(1), q_use & 1, abort_flag)) goto done;
+            const int qset = T::kQBufs == 4 ? (int)(k & 1) : 0;
+            if (!role_wait(b.q_full(2 * qset), q_use[qset] & 1, abort_flag)) goto done;
+            if (!role_wait(b.q_full(2 * qset + 1), q_use[qset] & 1, abort_flag)) goto done;
             tc_fence_after_sync();
             // S_t(i) into the next buffer in rotation; Q_t is released after its last product
             auto issue_s = [&](int t, int i, uint32_t kslot) {
                 const uint32_t col = (s_issued++ % 3) * 128;
-                fwd_issue_s<D, FP8>(tbase + col, dq0 + t * kTileStep, dk0 + kslot * kTileStep,
-                                    leader);
+                fwd_issue_s<D, FP8>(tbase + col, dq0 + (2 * qset + t) * kTileStep,
+                                    dk0 + kslot * kTileStep, leader);
                 mma_commit_w(b.template s_bar<3>(t, s_cnt[t]++), leader);
-                if (i == x.n[t] - 1) mma_commit_w(b.q_empty(t), leader);
+                if (i == x.n[t] - 1) mma_commit_w(b.q_empty(2 * qset + t), leader);
                 return col;
             };
             if (x.nmax > 0) {
@@ -586,8 +617,8 @@ __device__ void fwd_mma_ahead(const FwdParams& p, uint32_t tbase, uint32_t sQ, u
             }
             // Q tiles without any S product in this unit are released here
             for (int t = 0; t < 2; ++t)
-                if (x.n[t] == 0) mma_commit_w(b.q_empty(t), leader);
-            ++q_use;
+                if (x.n[t] == 0) mma_commit_w(b.q_empty(2 * qset + t), leader);
+            ++q_use[qset];
             for (int t = 0; t < 2; ++t)
                 if (x.n[t] > 0) ++o_use[t];
         }
@@ -612,15 +643,18 @@ __device__ void fwd_mma(const FwdParams& p, uint32_t tbase, uint32_t sQ, uint32_
     const uint64_t dv0 = fwd_sdesc<T>(sKV, T::kPanelBytes);           // MN-major V tile
     const uint32_t colS[2] = {T::kColS0, T::kColS1};
     const uint32_t colO[2] = {T::kColO0, T::kColO1};
-    uint32_t kv_iter = 0, q_use = 0;
+    uint32_t kv_iter = 0;
+    uint32_t q_use[2] = {0, 0};     // units that used Q set 0 / set 1
     uint32_t o_use[2] = {0, 0}, p_phase[2] = {0, 0};
     for (uint32_t k = 0;; ++k) {
         int u;
-        if (!fwd_next_unit(b, k, true, abort_flag, &u)) goto done;
+        if (!fwd_next_unit(p, b, k, true, abort_flag, &u)) goto done;
         if (u < 0) break;
         const FwdUnit x = fwd_unit<CAUSAL>(u, p);
-        if (!role_wait(b.q_full(0), q_use & 1, abort_flag)) goto done;
-        if (!role_wait(b.q_full(1), q_use & 1, abort_flag)) goto done;
+        const int qset = T::kQBufs == 4 ? (int)(k & 1) : 0;
+        const uint64_t dqs = dq0 + 2 * qset * kTileStep;
+        if (!role_wait(b.q_full(2 * qset), q_use[qset] & 1, abort_flag)) goto done;
+        if (!role_wait(b.q_full(2 * qset + 1), q_use[qset] & 1, abort_flag)) goto done;
         tc_fence_after_sync();
         if (x.nmax > 0) {
             uint32_t kslot = kv_iter % T::kSlots;
@@ -628,11 +662,11 @@ __device__ void fwd_mma(const FwdParams& p, uint32_t tbase, uint32_t sQ, uint32_
             tc_fence_after_sync();
             for (int t = 0; t < 2; ++t)
                 if (x.n[t] > 0) {
-                    fwd_issue_s<D, FP8>(tbase + colS[t], dq0 + t * kTileStep, dk0 + kslot * kTileStep,
+                    fwd_issue_s<D, FP8>(tbase + colS[t], dqs + t * kTileStep, dk0 + kslot * kTileStep,
                                    leader);
                     mma_commit_w(b.s_full(t), leader);
                     // Q_t's last use in this unit: let the producer refill it now
-                    if (x.n[t] == 1) mma_commit_w(b.q_empty(t), leader);
+                    if (x.n[t] == 1) mma_commit_w(b.q_empty(2 * qset + t), leader);
                 }
             mma_commit_w(b.kv_empty(kslot), leader);
             ++kv_iter;
@@ -672,10 +706,10 @@ __device__ void fwd_mma(const FwdParams& p, uint32_t tbase, uint32_t sQ, uint32_
                     }
                     if (t == 1) mma_commit_w(b.kv_empty(vslot), leader);
                     if (j + 1 < x.n[t]) {
-                        fwd_issue_s<D, FP8>(tbase + colS[t], dq0 + t * kTileStep,
+                        fwd_issue_s<D, FP8>(tbase + colS[t], dqs + t * kTileStep,
                                        dk0 + kslot * kTileStep, leader);
                         mma_commit_w(b.s_full(t), leader);
-                        if (j + 2 == x.n[t]) mma_commit_w(b.q_empty(t), leader);
+                        if (j + 2 == x.n[t]) mma_commit_w(b.q_empty(2 * qset + t), leader);
                     }
                 }
                 if (has_next) {
@@ -686,8 +720,8 @@ __device__ void fwd_mma(const FwdParams& p, uint32_t tbase, uint32_t sQ, uint32_
         }
         // Q tiles without any S product in this unit are released here
         for (int t = 0; t < 2; ++t)
-            if (x.n[t] == 0) mma_commit_w(b.q_empty(t), leader);
-        ++q_use;
+            if (x.n[t] == 0) mma_commit_w(b.q_empty(2 * qset + t), leader);
+        ++q_use[qset];
         for (int t = 0; t < 2; ++t)
             if (x.n[t] > 0) ++o_use[t];
     }
@@ -750,9 +784,9 @@ __device__ void fwd_softmax(const FwdParams& p, uint32_t tbase,
 
     for (uint32_t k = 0;; ++k) {
         int u;
-        const bool ok = fwd_next_unit(b, k, false, abort_flag, &u);
+        const bool ok = fwd_next_unit(p, b, k, false, abort_flag, &u);
         __syncwarp();
-        if (lane == 0 && ok) mbar_arrive(b.unit_empty(k & 1));
+        if (lane == 0 && ok && p.dynamic_units) mbar_arrive(b.unit_empty(k & 1));
         if (!__all_sync(0xffffffffu, ok)) return;
         if (u < 0) break;
         const FwdUnit x = fwd_unit<CAUSAL>(u, p);
@@ -942,10 +976,10 @@ __global__ void __launch_bounds__(384, 1)
     uint8_t* smem = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const uint32_t sQ = smem_addr(smem);
-    const uint32_t sKV = sQ + 2 * T::kTileBytes;
+    const uint32_t sKV = sQ + T::kQBufs * T::kTileBytes;
     // epilogue staging blocks, then the barriers (fwd_softmax finds its block
     // kStageBytes below the barrier base)
-    uint8_t* bar_ptr = smem + (2 + T::kSlots) * T::kTileBytes + T::kStageBytes;
+    uint8_t* bar_ptr = smem + (T::kQBufs + T::kSlots) * T::kTileBytes + T::kStageBytes;
     const uint32_t bar0 = smem_addr(bar_ptr);
     FwdBars<T::kSlots> b;
     b.base = bar0;
@@ -976,6 +1010,8 @@ __global__ void __launch_bounds__(384, 1)
             mbar_init(b.unit_empty(i), kUnitReaders);
             mbar_init(b.s_full_b(i), 1);
             mbar_init(b.pv_done(i), 1);
+            mbar_init(b.q_full(2 + i), 1);
+            mbar_init(b.q_empty(2 + i), 1);
         }
         *abort_flag = 0;
         fence_mbar_init();

@@ -122,9 +122,10 @@ struct FwdParams {
 #ifndef EATTN_SBUFS_AHEAD
 #define EATTN_SBUFS_AHEAD 1
 #endif
-// 1: two sets of Q tiles where shared memory allows (see FwdTraits::kQBufs)
+// 1: two sets of Q tiles where shared memory allows (see FwdTraits::kQBufs).
+//    Measured slower on gpt2_1k (45.1 against 43.0 us), so off.
 #ifndef EATTN_Q_DOUBLE
-#define EATTN_Q_DOUBLE 1
+#define EATTN_Q_DOUBLE 0
 #endif
 // 1: the epilogue's O stores go through shared memory as row-contiguous
 //    64-byte pieces (full sectors); 0: each thread stores its own row.
@@ -177,7 +178,7 @@ struct FwdTraits {
     static constexpr int kNumBars = 2 * kSlots + 27;   // FwdBars<kSlots>::kCount
     // epilogue staging: one 32-row x 64-byte (32 bf16 columns) block per softmax warp
     static constexpr int kStageWarpBytes = 32 * 64;
-    static constexpr int kStageBytes = 8 * kStageWarpBytes;
+    static constexpr int kStageBytes = EATTN_STAGE_O ? 8 * kStageWarpBytes : 0;
     // Q tiles: two (one unit's), or four where shared memory allows (head dim
     // 64, and e4m3 inputs), so that the next unit's Q is loaded while this
     // unit still runs instead of after its last S product
@@ -261,12 +262,17 @@ struct FwdUnit {
 template <bool CAUSAL>
 __device__ __forceinline__ FwdUnit fwd_unit(int u, const FwdParams& p) {
     FwdUnit x;
-    const int per_group = p.group_heads * p.num_qb;
-    const int g = u / per_group;
-    const int r = u - g * per_group;
-    const int heads = min(p.group_heads, p.BH - g * p.group_heads);   // the last group may be short
-    x.qb = p.num_qb - 1 - r / heads;   // heaviest (latest) query blocks first
-    x.bh = g * p.group_heads + r % heads;
+    if (p.group_heads >= p.BH) {   // one group: plain heaviest-first order
+        x.qb = p.num_qb - 1 - u / p.BH;
+        x.bh = u % p.BH;
+    } else {
+        const int per_group = p.group_heads * p.num_qb;
+        const int g = u / per_group;
+        const int r = u - g * per_group;
+        const int heads = min(p.group_heads, p.BH - g * p.group_heads);   // the last group may be short
+        x.qb = p.num_qb - 1 - r / heads;   // heaviest (latest) query blocks first
+        x.bh = g * p.group_heads + r % heads;
+    }
     dcheck(x.qb >= 0 && x.bh < p.BH);
 #pragma unroll
     for (int t = 0; t < 2; ++t) {

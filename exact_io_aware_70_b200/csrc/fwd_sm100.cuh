@@ -937,25 +937,16 @@ __device__ void fwd_softmax(const FwdParams& p, uint32_t tbase,
             uint16_t* o_rows = p.o + ((size_t)x.bh * p.Nq + (size_t)max(row0, 0)) * D;
             // the staging blocks sit right below the barriers
             const uint32_t stage = b.base - T::kStageBytes + warp * T::kStageWarpBytes;
-            // all of this row's O in one TMEM round trip; the tile's TMEM columns
-            // are free again as soon as it is in registers
-            uint32_t orr[D];
-            if constexpr (D == 128) {
-                tmem_ld128(tO, orr);
-                tmem_wait_ld128(orr);
-            } else {
-                tmem_ld64(tO, orr);
-                tmem_wait_ld64(orr);
-            }
-            tc_fence_before_sync();
-            mbar_arrive(bar_ofree);
-#pragma unroll
+#pragma unroll 1
             for (int c = 0; c < D; c += 32) {
+                uint32_t orr[32];
+                tmem_ld32(tO + c, orr);
+                tmem_wait_ld(orr);
                 uint32_t w[16];
 #pragma unroll
                 for (int i = 0; i < 16; ++i)
-                    w[i] = pack_bf16x2(__uint_as_float(orr[c + 2 * i]) * inv,
-                                       __uint_as_float(orr[c + 2 * i + 1]) * inv);
+                    w[i] = pack_bf16x2(__uint_as_float(orr[2 * i]) * inv,
+                                       __uint_as_float(orr[2 * i + 1]) * inv);
                 if (EATTN_STAGE_O) {
                     fwd_store_chunk<D>(stage, w, lane, o_rows, c, valid_rows,
                                        p.o + (size_t)p.BH * p.Nq * D);
@@ -966,6 +957,8 @@ __device__ void fwd_softmax(const FwdParams& p, uint32_t tbase,
                         dst[k4] = make_uint4(w[4 * k4], w[4 * k4 + 1], w[4 * k4 + 2], w[4 * k4 + 3]);
                 }
             }
+            tc_fence_before_sync();
+            mbar_arrive(bar_ofree);
             ++o_use;
         } else if (row_valid && dcheck(x.bh < p.BH)) {
             uint4* dst = reinterpret_cast<uint4*>(orow);

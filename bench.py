@@ -265,7 +265,7 @@ class ClockSampler:
 KERNEL_SOURCES = {
     "attn_fwd_sm100": ("fwd_sm100.cuh", "ptx_sm100.cuh", "tmem_wide.cuh"),
     "attn_decode_partials": ("decode_sm100.cuh", "ptx_sm100.cuh"),
-    "attn_lse_merge": ("decode_sm100.cuh",),
+    "attn_lse_merge": ("decode_sm100.cuh", "ptx_sm100.cuh"),
     "attn_bwd_sm100": ("bwd_sm100.cuh", "ptx_sm100.cuh", "tmem_wide.cuh"),
     "attn_fwd_sm100_e4m3": ("fwd_sm100.cuh", "ptx_sm100.cuh", "tmem_wide.cuh"),
 }
@@ -288,7 +288,8 @@ def kernel_source_hash(kernel):
 
 def recorded_traffic():
     """Per-launch DRAM traffic from the committed ncu summary, for each kernel
-    whose sources still hash to the value recorded with its figure."""
+    whose sources still hash to the value recorded with its figure, keyed by
+    (kernel name, workload)."""
     path = os.path.join(ROOT, "profiles", "dram_traffic.md")
     try:
         with open(path) as fh:
@@ -301,7 +302,7 @@ def recorded_traffic():
             r"^\|\s*(attn_\w+)\s*\|\s*([\w ]+?)\s*\|\s*(\d+)\s*\|\s*([0-9a-f]{16})\s*\|",
             text, re.M):
         if name in KERNEL_SOURCES and shash == kernel_source_hash(name):
-            out[name] = int(nbytes)
+            out[(name, _wl)] = int(nbytes)
     return out
 
 
@@ -628,7 +629,7 @@ def run_fp8(args):
             "peak": fp8_peak, "unit": "TFLOP/s", "frac": a / fp8_peak,
             "peak_note": "measured bf16 peak x 2 (nominal e4m3 / bf16 dense ratio)",
             "frac_of_bf16_peak": a / pk["bf16_tflops"],
-            "traffic": recorded_traffic().get("attn_fwd_sm100_e4m3"),
+            "traffic": recorded_traffic().get(("attn_fwd_sm100_e4m3", args.workload)),
             "algorithmic_bytes": prefill_bytes(w) // 2 + w.B * w.H * w.Nq * w.d,
             "algorithmic_flops": prefill_flops(w), "ms": call_ms}
     line = {
@@ -755,7 +756,7 @@ def run_bwd(args):
     roof = {"kernel": "attn_bwd (preprocess + attn_bwd_sm100 + postprocess, timed as one call)",
             "bound": "tensor", "achieved": a, "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
             "frac": a / pk["bf16_tflops"], "frac_of_sustained": a / pk["bf16_tflops_sustained"],
-            "traffic": recorded_traffic().get("attn_bwd_sm100"),
+            "traffic": recorded_traffic().get(("attn_bwd_sm100", args.workload)),
             "algorithmic_bytes": bwd_bytes(w), "algorithmic_flops": bwd_flops(w), "ms": call_ms}
     line = {
         "metric": "attn bwd TFLOP/s & % BF16 tensor peak",
@@ -841,7 +842,9 @@ def time_prefill_workload(ea, w, K, warmup, dev, stream, local, cpu_budget):
     out = {"config": {"B": w.B, "H": w.H, "N": w.Nq, "d": w.d, "causal": w.causal,
                       "seed": w.seed, "l2": flush.note},
            "ms": call_ms, "value": prefill_flops(w) / (call_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
-           "roofline": dict(prefill_roofline(w, call_ms, pk), kernel="attn_fwd_sm100"),
+           "roofline": dict(prefill_roofline(w, call_ms, pk,
+                                             recorded_traffic().get(("attn_fwd_sm100", w.name))),
+                            kernel="attn_fwd_sm100"),
            "clocks": clk.summary(max_mhz_default=1965.0), "gpu_launches": K}
     if hot_ms is not None:
         out["hot"] = {"ms": hot_ms, "value": prefill_flops(w) / (hot_ms * 1e-3) / 1e12,
@@ -1112,7 +1115,7 @@ def run_ours(args):
     roof = {}
     if pw:
         roof["attn_fwd_sm100"] = dict(prefill_roofline(pw, kms["attn_fwd_sm100"], pk,
-                                                       traffic.get("attn_fwd_sm100")),
+                                                       traffic.get(("attn_fwd_sm100", pw.name))),
                                       share=kms["attn_fwd_sm100"] / step_ms)
     if dw:
         mbytes = merge_bytes(dw) * ws
@@ -1121,7 +1124,7 @@ def run_ours(args):
             t = kms[name]
             a = nbytes / (t * 1e-3) / 1e9
             roof[name] = {"bound": "hbm", "achieved": a, "peak": pk["hbm_gbs"], "unit": "GB/s",
-                          "frac": a / pk["hbm_gbs"], "traffic": traffic.get(name),
+                          "frac": a / pk["hbm_gbs"], "traffic": traffic.get((name, dw.name)),
                           "algorithmic_bytes": nbytes, "ms": t, "share": t / step_ms,
                           "note": _peaks_note(pk)}
     dominant = max(roof, key=lambda n: roof[n]["ms"])

@@ -34,8 +34,8 @@ def test_decode_bytes_model():
 
 def test_recorded_traffic_needs_matching_source_hash(monkeypatch):
     good = bench.recorded_traffic()
-    for name, nbytes in good.items():
-        assert name in bench.KERNEL_SOURCES and nbytes > 0
+    for (name, workload), nbytes in good.items():
+        assert name in bench.KERNEL_SOURCES and workload and nbytes > 0
     monkeypatch.setattr(bench, "kernel_source_hash", lambda kernel: "0000000000000000")
     assert bench.recorded_traffic() == {}
 

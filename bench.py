@@ -924,8 +924,11 @@ def run_ours(args):
                 dq = make_paged_cache(dw.B, dw.H, [dw.Nkv] * dw.B, dw.d, PD["page_size"],
                                       dw.seed, device="cuda")[0]
         else:
-            _, dk, dv = make_workload(dw_r, device="cuda")
-            dq = make_workload(dw, device="cuda")[0] if ws > 1 else make_workload(dw_r, "cuda")[0]
+            dq, dk, dv = make_workload(dw_r, device="cuda")
+            if ws > 1:
+                # the query rows are the same on every rank (the base seed's first draw,
+                # which does not depend on the key count); the keys are the rank's shard
+                dq = make_qkv(dw.B, dw.H, 1, 1, dw.d, dw.seed, device="cuda")[0]
         do = torch.empty_like(dq)
         dlse = torch.empty((dw.B, dw.H, 1), dtype=torch.float32, device=dev)
         work = torch.empty(ea.attn_decode_workspace_bytes(dw.B, dw.H, dw.d, S), dtype=torch.uint8,

@@ -131,3 +131,13 @@ def test_kv_split_decode_on_gloo_ranks_equals_unsplit(world, Nkv, S):
         assert dec_err[0] <= 1e-12 and dec_err[1] <= 1e-12, dec_err
         assert pf_err == 0.0
         assert t == [float(world), 5.0]                 # element-wise max over ranks
+
+
+def test_query_draw_does_not_depend_on_the_key_count():
+    """Every rank of the split decode draws the same query rows from the base
+    seed without drawing the whole sequence's keys: the queries are the
+    generator's first draw, so they do not depend on how many keys follow."""
+    from seeded_inputs import make_qkv
+    q_small = make_qkv(2, 3, 1, 1, 16, seed=4)[0]
+    q_full = make_qkv(2, 3, 1, 4097, 16, seed=4)[0]
+    assert torch.equal(q_small, q_full)

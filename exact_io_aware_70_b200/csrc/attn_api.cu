@@ -141,6 +141,10 @@ int fwd_group_heads(int BH, int Nkv, int d, int elem_bytes) {
 // heads exceed this (the launch's K/V then cannot stay in the 126 MB L2 while
 // every head is in flight); below it a static deal of the heaviest-first
 // order is used. 0 forces the dynamic queue, a huge value the static deal.
+// 1: the static deal also walks the units in head groups (measured slower)
+#ifndef EATTN_FWD_STATIC_GROUPS
+#define EATTN_FWD_STATIC_GROUPS 0
+#endif
 #ifndef EATTN_FWD_QUEUE_MIN_BYTES
 #define EATTN_FWD_QUEUE_MIN_BYTES (192ll << 20)
 #endif
@@ -177,7 +181,9 @@ attn_status_t launch_fwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUt
         if (std::strcmp(sched, "dynamic") == 0) p.dynamic_units = 1;
         if (std::strcmp(sched, "static") == 0) p.dynamic_units = 0;
     }
-    p.group_heads = p.dynamic_units ? fwd_group_heads(p.BH, p.Nkv, D, T::kElemBytes) : p.BH;
+    p.group_heads = (p.dynamic_units || EATTN_FWD_STATIC_GROUPS)
+                        ? fwd_group_heads(p.BH, p.Nkv, D, T::kElemBytes)
+                        : p.BH;
     p.queue_slot = (int)(g_fwd_queue_rr.fetch_add(1, std::memory_order_relaxed) % kFwdQueueSlots);
     kern<<<grid, T::kThreads, T::kSmemBytes, stream>>>(tq, tk, tv, p);
     return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;

@@ -127,6 +127,11 @@ struct FwdParams {
 #ifndef EATTN_Q_DOUBLE
 #define EATTN_Q_DOUBLE 0
 #endif
+// 1: the O stores carry an evict-first L2 policy (O is written once and not
+//    read again by this kernel), so they do not push K/V tiles out of L2.
+#ifndef EATTN_O_EVICT_FIRST
+#define EATTN_O_EVICT_FIRST 0
+#endif
 // 1: the epilogue's O stores go through shared memory as row-contiguous
 //    64-byte pieces (full sectors); 0: each thread stores its own row.
 #ifndef EATTN_STAGE_O
@@ -768,7 +773,12 @@ __device__ __forceinline__ void fwd_store_chunk(uint32_t stage, const uint32_t (
         const int r = i * 8 + (lane >> 2), k = lane & 3;
         const uint4 val = ld_shared_v4(stage + stage_slot(r, k));
         uint16_t* dst = o_rows + (size_t)r * D + c + 8 * k;
-        if (r < valid_rows && dcheck(dst + 8 <= o_end)) *reinterpret_cast<uint4*>(dst) = val;
+        if (r < valid_rows && dcheck(dst + 8 <= o_end)) {
+            if (EATTN_O_EVICT_FIRST)
+                st_global_v4_hint(dst, val, l2_policy_evict_first());
+            else
+                *reinterpret_cast<uint4*>(dst) = val;
+        }
     }
 }
 

@@ -127,10 +127,10 @@ struct FwdParams {
 #ifndef EATTN_Q_DOUBLE
 #define EATTN_Q_DOUBLE 0
 #endif
-// 1: the O stores carry an evict-first L2 policy (O is written once and not
-//    read again by this kernel), so they do not push K/V tiles out of L2.
-#ifndef EATTN_O_EVICT_FIRST
-#define EATTN_O_EVICT_FIRST 0
+// Row max over a score tile: 4 chains of three-input maxima (4), or 16 chains
+// and a tree (16).
+#ifndef EATTN_MAX_CHAINS
+#define EATTN_MAX_CHAINS 4
 #endif
 // 1: the epilogue's O stores go through shared memory as row-contiguous
 //    64-byte pieces (full sectors); 0: each thread stores its own row.
@@ -773,12 +773,7 @@ __device__ __forceinline__ void fwd_store_chunk(uint32_t stage, const uint32_t (
         const int r = i * 8 + (lane >> 2), k = lane & 3;
         const uint4 val = ld_shared_v4(stage + stage_slot(r, k));
         uint16_t* dst = o_rows + (size_t)r * D + c + 8 * k;
-        if (r < valid_rows && dcheck(dst + 8 <= o_end)) {
-            if (EATTN_O_EVICT_FIRST)
-                st_global_v4_hint(dst, val, l2_policy_evict_first());
-            else
-                *reinterpret_cast<uint4*>(dst) = val;
-        }
+        if (r < valid_rows && dcheck(dst + 8 <= o_end)) *reinterpret_cast<uint4*>(dst) = val;
     }
 }
 
@@ -841,15 +836,36 @@ __device__ void fwd_softmax(const FwdParams& p, uint32_t tbase,
                         if (c >= lim) sr[c] = __float_as_uint(-INFINITY);
                 }
             }
-            float mx0 = -INFINITY, mx1 = -INFINITY, mx2 = -INFINITY, mx3 = -INFINITY;
+            float mxs;
+            if (EATTN_MAX_CHAINS == 16) {
+                // 16 independent chains of 4 three-input maxima, then a small tree:
+                // a dependent depth of 7 instead of 18
+                float mc[16];
 #pragma unroll
-            for (int c = 0; c < 128; c += 8) {
-                mx0 = fmax3(mx0, __uint_as_float(sr[c]), __uint_as_float(sr[c + 1]));
-                mx1 = fmax3(mx1, __uint_as_float(sr[c + 2]), __uint_as_float(sr[c + 3]));
-                mx2 = fmax3(mx2, __uint_as_float(sr[c + 4]), __uint_as_float(sr[c + 5]));
-                mx3 = fmax3(mx3, __uint_as_float(sr[c + 6]), __uint_as_float(sr[c + 7]));
+                for (int q = 0; q < 16; ++q)
+                    mc[q] = fmax3(__uint_as_float(sr[8 * q]), __uint_as_float(sr[8 * q + 1]),
+                                  __uint_as_float(sr[8 * q + 2]));
+#pragma unroll
+                for (int q = 0; q < 16; ++q) {
+                    mc[q] = fmax3(mc[q], __uint_as_float(sr[8 * q + 3]), __uint_as_float(sr[8 * q + 4]));
+                    mc[q] = fmax3(mc[q], __uint_as_float(sr[8 * q + 5]), __uint_as_float(sr[8 * q + 6]));
+                    mc[q] = fmaxf(mc[q], __uint_as_float(sr[8 * q + 7]));
+                }
+                const float a = fmax3(mc[0], mc[1], mc[2]), b2 = fmax3(mc[3], mc[4], mc[5]);
+                const float c3 = fmax3(mc[6], mc[7], mc[8]), d3 = fmax3(mc[9], mc[10], mc[11]);
+                const float e3 = fmax3(mc[12], mc[13], mc[14]);
+                mxs = fmax3(fmax3(a, b2, c3), fmax3(d3, e3, mc[15]), -INFINITY) * c2;
+            } else {
+                float mx0 = -INFINITY, mx1 = -INFINITY, mx2 = -INFINITY, mx3 = -INFINITY;
+#pragma unroll
+                for (int c = 0; c < 128; c += 8) {
+                    mx0 = fmax3(mx0, __uint_as_float(sr[c]), __uint_as_float(sr[c + 1]));
+                    mx1 = fmax3(mx1, __uint_as_float(sr[c + 2]), __uint_as_float(sr[c + 3]));
+                    mx2 = fmax3(mx2, __uint_as_float(sr[c + 4]), __uint_as_float(sr[c + 5]));
+                    mx3 = fmax3(mx3, __uint_as_float(sr[c + 6]), __uint_as_float(sr[c + 7]));
+                }
+                mxs = fmax3(mx0, mx1, fmaxf(mx2, mx3)) * c2;
             }
-            const float mxs = fmax3(mx0, mx1, fmaxf(mx2, mx3)) * c2;
             const bool need = mxs > m_ref + T::kLazy;
             const bool any_need = __any_sync(0xffffffffu, need);
             const float m_new = need ? mxs : m_ref;

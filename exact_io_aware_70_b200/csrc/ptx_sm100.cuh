@@ -62,13 +62,6 @@ __device__ __forceinline__ uint4 ld_shared_v4(uint32_t addr) {
     return r;
 }
 
-// 16-byte global store with an L2 cache policy (from createpolicy)
-__device__ __forceinline__ void st_global_v4_hint(void* p, uint4 v, uint64_t pol) {
-    asm volatile("st.global.L2::cache_hint.v4.b32 [%0], {%1, %2, %3, %4}, %5;" ::"l"(p),
-                 "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w), "l"(pol)
-                 : "memory");
-}
-
 __device__ __forceinline__ unsigned long long global_timer_ns() {
     unsigned long long t;
     asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));

@@ -127,11 +127,6 @@ struct FwdParams {
 #ifndef EATTN_Q_DOUBLE
 #define EATTN_Q_DOUBLE 0
 #endif
-// Row max over a score tile: 4 chains of three-input maxima (4), or 16 chains
-// and a tree (16).
-#ifndef EATTN_MAX_CHAINS
-#define EATTN_MAX_CHAINS 4
-#endif
 // 1: the epilogue's O stores go through shared memory as row-contiguous
 //    64-byte pieces (full sectors); 0: each thread stores its own row.
 #ifndef EATTN_STAGE_O
@@ -836,36 +831,15 @@ __device__ void fwd_softmax(const FwdParams& p, uint32_t tbase,
                         if (c >= lim) sr[c] = __float_as_uint(-INFINITY);
                 }
             }
-            float mxs;
-            if (EATTN_MAX_CHAINS == 16) {
-                // 16 independent chains of 4 three-input maxima, then a small tree:
-                // a dependent depth of 7 instead of 18
-                float mc[16];
+            float mx0 = -INFINITY, mx1 = -INFINITY, mx2 = -INFINITY, mx3 = -INFINITY;
 #pragma unroll
-                for (int q = 0; q < 16; ++q)
-                    mc[q] = fmax3(__uint_as_float(sr[8 * q]), __uint_as_float(sr[8 * q + 1]),
-                                  __uint_as_float(sr[8 * q + 2]));
-#pragma unroll
-                for (int q = 0; q < 16; ++q) {
-                    mc[q] = fmax3(mc[q], __uint_as_float(sr[8 * q + 3]), __uint_as_float(sr[8 * q + 4]));
-                    mc[q] = fmax3(mc[q], __uint_as_float(sr[8 * q + 5]), __uint_as_float(sr[8 * q + 6]));
-                    mc[q] = fmaxf(mc[q], __uint_as_float(sr[8 * q + 7]));
-                }
-                const float a = fmax3(mc[0], mc[1], mc[2]), b2 = fmax3(mc[3], mc[4], mc[5]);
-                const float c3 = fmax3(mc[6], mc[7], mc[8]), d3 = fmax3(mc[9], mc[10], mc[11]);
-                const float e3 = fmax3(mc[12], mc[13], mc[14]);
-                mxs = fmax3(fmax3(a, b2, c3), fmax3(d3, e3, mc[15]), -INFINITY) * c2;
-            } else {
-                float mx0 = -INFINITY, mx1 = -INFINITY, mx2 = -INFINITY, mx3 = -INFINITY;
-#pragma unroll
-                for (int c = 0; c < 128; c += 8) {
-                    mx0 = fmax3(mx0, __uint_as_float(sr[c]), __uint_as_float(sr[c + 1]));
-                    mx1 = fmax3(mx1, __uint_as_float(sr[c + 2]), __uint_as_float(sr[c + 3]));
-                    mx2 = fmax3(mx2, __uint_as_float(sr[c + 4]), __uint_as_float(sr[c + 5]));
-                    mx3 = fmax3(mx3, __uint_as_float(sr[c + 6]), __uint_as_float(sr[c + 7]));
-                }
-                mxs = fmax3(mx0, mx1, fmaxf(mx2, mx3)) * c2;
+            for (int c = 0; c < 128; c += 8) {
+                mx0 = fmax3(mx0, __uint_as_float(sr[c]), __uint_as_float(sr[c + 1]));
+                mx1 = fmax3(mx1, __uint_as_float(sr[c + 2]), __uint_as_float(sr[c + 3]));
+                mx2 = fmax3(mx2, __uint_as_float(sr[c + 4]), __uint_as_float(sr[c + 5]));
+                mx3 = fmax3(mx3, __uint_as_float(sr[c + 6]), __uint_as_float(sr[c + 7]));
             }
+            const float mxs = fmax3(mx0, mx1, fmaxf(mx2, mx3)) * c2;
             const bool need = mxs > m_ref + T::kLazy;
             const bool any_need = __any_sync(0xffffffffu, need);
             const float m_new = need ? mxs : m_ref;

@@ -75,6 +75,16 @@ int attn_abi_version(void);
  *   lse fp32 [B, H, Nq]         (written)
  *   d in {64, 128}; B, H, Nq, Nkv >= 1; causal 0 or 1; scale finite (usually
  *   1/sqrt(d)). Any Nq, Nkv is accepted; tails of a 128-row tile are masked.
+ *
+ *   Work is dealt to one persistent CTA per SM. When the K and V of all heads
+ *   exceed 192 MB, the CTAs take their work units from a counter in device
+ *   memory owned by the library (one of 64 entries, chosen round robin per
+ *   call and returned to zero by the launch itself), in an order that keeps a
+ *   few heads' K/V in L2. Two launches that run at the same time use
+ *   different entries unless 64 further launches start while the first still
+ *   runs; such launches would share an entry and give wrong results. The
+ *   environment variable EXACT_ATTN_FWD_SCHEDULE=static|dynamic, read at
+ *   every call, forces one deal or the other; the result is bit-identical.
  */
 attn_status_t attn_fwd(const void *q, const void *k, const void *v, void *o, float *lse,
                        int B, int H, int Nq, int Nkv, int d, int causal, float scale,
@@ -100,7 +110,8 @@ attn_status_t attn_fwd(const void *q, const void *k, const void *v, void *o, flo
  *   o                 bf16 [B, H, Nq, d]      (written)
  *   lse               fp32 [B, H, Nq]         (written; natural log, as attn_fwd)
  *   d in {64, 128} (ATTN_ERR_UNSUPPORTED otherwise); causal, scale and the
- *   size limits as attn_fwd; q, k, v, o 16-byte aligned, the rest 4-byte.
+ *   size limits and the work deal (K/V measured in bytes) as attn_fwd; q, k, v,
+ *   o 16-byte aligned, the rest 4-byte.
  */
 attn_status_t attn_fwd_fp8(const void *q, const void *k, const void *v, const float *q_descale,
                            const float *k_descale, const float *v_descale, void *o, float *lse,

@@ -122,11 +122,6 @@ struct FwdParams {
 #ifndef EATTN_SBUFS_AHEAD
 #define EATTN_SBUFS_AHEAD 1
 #endif
-// 1: each unit reads the K/V tiles its two Q tiles share starting at a
-//    per-unit offset (fwd_kv_tile); 0: in order from tile 0.
-#ifndef EATTN_KV_ROTATE
-#define EATTN_KV_ROTATE 0
-#endif
 // 1: two sets of Q tiles where shared memory allows (see FwdTraits::kQBufs).
 //    Measured slower on gpt2_1k (45.1 against 43.0 us), so off.
 #ifndef EATTN_Q_DOUBLE
@@ -262,21 +257,7 @@ struct FwdUnit {
     int bh, qb;
     int n[2];   // K/V tiles visible to Q tile 0 / Q tile 1 (0: tile has no work)
     int nmax;
-    int rot;    // K/V tile order: step j < n[0] reads tile (j + rot) mod n[0]
 };
-
-// The K/V tile a unit reads at step j. Both Q tiles share the tiles every
-// step, and tile 0 stops after n[0] steps, so the tiles both need come first
-// and the one or more only tile 1 sees come last, in order; the shared ones
-// start at a per-unit offset, so that CTAs working on the same head at the
-// same moment read different tiles rather than all the same one. The online
-// softmax does not depend on the order (the causal mask goes by the absolute
-// tile index).
-__device__ __forceinline__ int fwd_kv_tile(const FwdUnit& x, int j) {
-    if (j >= x.n[0] || x.rot == 0) return j;
-    const int t = j + x.rot;
-    return t >= x.n[0] ? t - x.n[0] : t;
-}
 
 template <bool CAUSAL>
 __device__ __forceinline__ FwdUnit fwd_unit(int u, const FwdParams& p) {
@@ -308,10 +289,6 @@ __device__ __forceinline__ FwdUnit fwd_unit(int u, const FwdParams& p) {
         x.n[t] = n;
     }
     x.nmax = max(x.n[0], x.n[1]);
-    // a spread of offsets over the units of one head (golden-ratio steps)
-    x.rot = (EATTN_KV_ROTATE && x.n[0] > 1)
-                ? (int)(((unsigned)(x.qb * 2654435761u + x.bh * 40503u) >> 16) % (unsigned)x.n[0])
-                : 0;
     return x;
 }
 
@@ -475,13 +452,11 @@ __device__ void fwd_producer(const FwdParams& p, const CUtensorMap* tq, const CU
                 for (int pn = 0; pn < T::kPanels; ++pn)
                     if (EATTN_FWD_L2_HINTS)
                         tma_load_3d_hint_w(sKV + slot * T::kTileBytes + pn * T::kPanelBytes,
-                                           which ? tv : tk, fbar, pn * T::kPanelElems,
-                                           fwd_kv_tile(x, j) * 128,
+                                           which ? tv : tk, fbar, pn * T::kPanelElems, j * 128,
                                            x.bh, pol_kv, leader);
                     else
                         tma_load_3d_w(sKV + slot * T::kTileBytes + pn * T::kPanelBytes,
-                                      which ? tv : tk, fbar, pn * T::kPanelElems,
-                                      fwd_kv_tile(x, j) * 128, x.bh,
+                                      which ? tv : tk, fbar, pn * T::kPanelElems, j * 128, x.bh,
                                       leader);
                 ++kv_iter;
             }
@@ -849,7 +824,7 @@ __device__ void fwd_softmax(const FwdParams& p, uint32_t tbase,
             tmem_wait_ld128(sr);
             {
                 // columns c >= lim of this tile are masked (-inf) for this row
-                const int lim = max(-1, min(128, kv_lim - fwd_kv_tile(x, j) * 128));
+                const int lim = max(-1, min(128, kv_lim - j * 128));
                 if (lim < 128) {
 #pragma unroll
                     for (int c = 0; c < 128; ++c)

@@ -122,17 +122,6 @@ struct FwdParams {
 #ifndef EATTN_SBUFS_AHEAD
 #define EATTN_SBUFS_AHEAD 1
 #endif
-// 1: (bf16) the softmax exponentiates and stores P in four parts of 32 columns
-//    instead of two of 64
-#ifndef EATTN_SM_QUARTERS
-#define EATTN_SM_QUARTERS 0
-#endif
-static_assert(!(EATTN_SM_QUARTERS && EATTN_SPLIT_P), "P is handed over once per step in parts");
-// 1: P (non-negative) is packed to bf16 with integer instructions, rounding
-//    half up; 0: cvt.rn.bf16x2.f32 (round to nearest even).
-#ifndef EATTN_P_PACK_INT
-#define EATTN_P_PACK_INT 0
-#endif
 // 1: two sets of Q tiles where shared memory allows (see FwdTraits::kQBufs).
 //    Measured slower on gpt2_1k (45.1 against 43.0 us), so off.
 #ifndef EATTN_Q_DOUBLE
@@ -861,16 +850,12 @@ __device__ void fwd_softmax(const FwdParams& p, uint32_t tbase,
             const f32x2_t nbx2 = f2_pack(-base, -base);
             f32x2_t lsum_a = f2_pack(0.f, 0.f), lsum_b = f2_pack(0.f, 0.f);
 #pragma unroll
-            // the row in kParts parts of 128 / kParts columns, each stored to TMEM as
-            // P as soon as it is exponentiated
-            constexpr int kParts = (EATTN_SM_QUARTERS && !FP8) ? 4 : 2;
-            constexpr int kPairs = 64 / kParts;
-            for (int h = 0; h < kParts; ++h) {
-                uint32_t pk[FP8 ? kPairs / 2 : kPairs];     // bf16 pairs or e4m3 quads
+            for (int h = 0; h < 2; ++h) {
+                uint32_t pk[FP8 ? 16 : 32];     // bf16 pairs or e4m3 quads
                 float e_prev0 = 0.f, e_prev1 = 0.f;
 #pragma unroll
-                for (int i = 0; i < kPairs; ++i) {
-                    const int c = 2 * kPairs * h + 2 * i;
+                for (int i = 0; i < 32; ++i) {
+                    const int c = 64 * h + 2 * i;
                     const f32x2_t xv = f2_fma(
                         f2_pack(__uint_as_float(sr[c]), __uint_as_float(sr[c + 1])), c2x2, nbx2);
                     float e0, e1;
@@ -884,7 +869,7 @@ __device__ void fwd_softmax(const FwdParams& p, uint32_t tbase,
                         e1 = fast_exp2(x1);
                     }
                     if constexpr (!FP8) {
-                        pk[i] = EATTN_P_PACK_INT ? pack_bf16x2_pos(e0, e1) : pack_bf16x2(e0, e1);
+                        pk[i] = pack_bf16x2(e0, e1);
                     } else if (i & 1) {
                         pk[i / 2] = pack_e4m3x4(e_prev0, e_prev1, e0, e1);
                     } else {
@@ -920,11 +905,9 @@ __device__ void fwd_softmax(const FwdParams& p, uint32_t tbase,
                 }
                 if constexpr (FP8)
                     tmem_st16(tS + 16 * h, pk);
-                else if constexpr (kParts == 4)
-                    tmem_st16(tS + 16 * h, pk);
                 else
                     tmem_st32(tS + 32 * h, pk);
-                if (EATTN_SPLIT_P || h == kParts - 1) {
+                if (EATTN_SPLIT_P || h == 1) {
                     tmem_wait_st();
                     tc_fence_before_sync();
                     // three score buffers: P_t tiles alternate between p_hi and p_lo

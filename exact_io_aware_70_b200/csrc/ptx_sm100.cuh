@@ -520,14 +520,6 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     return r;
 }
 
-// Two non-negative finite fp32 -> packed bf16x2 with integer instructions
-// (add half a bf16 unit in the last place, keep the upper 16 bits; PRMT packs
-// the two upper halves): round half up, which for these values differs from
-// round to nearest even only on exact ties. `lo` lands in bits 0-15.
-__device__ __forceinline__ uint32_t pack_bf16x2_pos(float lo, float hi) {
-    return __byte_perm(__float_as_uint(lo) + 0x8000u, __float_as_uint(hi) + 0x8000u, 0x7632);
-}
-
 // Four fp32 -> four e4m3 in one word (round to nearest even, saturating to
 // +-448); `a` lands in bits 0-7, `d` in bits 24-31 (lowest K index lowest).
 __device__ __forceinline__ uint32_t pack_e4m3x4(float a, float b, float c, float d) {

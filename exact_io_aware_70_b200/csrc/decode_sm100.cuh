@@ -92,12 +92,22 @@ __device__ __forceinline__ void axpy8(float p, const uint4& kv, float (&acc)[8])
     acc[7] = fmaf(p, bf16_hi(kv.w), acc[7]);
 }
 
+// 16-byte K (then V) rows each thread has in flight per pass, and the
+// minimum resident CTAs per SM the contiguous kernel is compiled for.
+#ifndef EATTN_DECODE_BATCH
+#define EATTN_DECODE_BATCH 8
+#endif
+#ifndef EATTN_DECODE_MIN_CTAS
+#define EATTN_DECODE_MIN_CTAS 1
+#endif
+
 template <int D>
 struct DecodeTraits {
     static constexpr int kThreads = 256;
     static constexpr int kLanesPerRow = D / 8;                     // 16-byte pieces per row
     static constexpr int kRowsPerPass = kThreads / kLanesPerRow;   // rows covered by one load of all threads
-    static constexpr int kBatch = 8;                               // rows in flight per thread
+    static constexpr int kBatch = EATTN_DECODE_BATCH;              // rows in flight per thread
+    static_assert(kBatch % 8 == 0, "the score pass reduces rows in groups of 8");
     static constexpr int kSub = kRowsPerPass * kBatch * 4;         // keys per sub-block
 };
 
@@ -155,7 +165,7 @@ __device__ __forceinline__ int reduce_owner_index(int glane) {
 // The paged instantiation is held to 64 registers (4 CTAs per SM): measured
 // 6.63 TB/s against 4.83 TB/s at its unconstrained 80 registers (3 CTAs).
 template <int D, bool PAGED>
-__global__ void __launch_bounds__(256, PAGED ? 4 : 1)
+__global__ void __launch_bounds__(256, PAGED ? 4 : EATTN_DECODE_MIN_CTAS)
     attn_decode_partials_kernel(const DecodeParams p) {
     using T = DecodeTraits<D>;
     constexpr int LPR = T::kLanesPerRow, RPP = T::kRowsPerPass, NB = T::kBatch;
@@ -259,17 +269,21 @@ __global__ void __launch_bounds__(256, PAGED ? 4 : 1)
                                 : make_uint4(0, 0, 0, 0);
                 }
             }
-            float part[8];
+            // the transpose-reduce sums 8 rows at a time
 #pragma unroll
-            for (int r = 0; r < NB; ++r) part[r] = dot8(kr[r], qv);
-            const float sum = group_transpose_reduce8<LPR>(part, glane);
-            const int owner = reduce_owner_index<D>(glane);
-            const bool writer = (LPR == 16) ? ((glane & 1) == 0) : true;
-            if (writer) {
-                const int i = base + rs + RPP * owner;
-                bool skipped = i >= nsub;
-                if (PAGED && !skipped) skipped = page_of(sb + i, lp0) < 0;
-                s_score[i] = skipped ? -INFINITY : sum;
+            for (int g = 0; g < NB / 8; ++g) {
+                float part[8];
+#pragma unroll
+                for (int r = 0; r < 8; ++r) part[r] = dot8(kr[8 * g + r], qv);
+                const float sum = group_transpose_reduce8<LPR>(part, glane);
+                const int owner = 8 * g + reduce_owner_index<D>(glane);
+                const bool writer = (LPR == 16) ? ((glane & 1) == 0) : true;
+                if (writer) {
+                    const int i = base + rs + RPP * owner;
+                    bool skipped = i >= nsub;
+                    if (PAGED && !skipped) skipped = page_of(sb + i, lp0) < 0;
+                    s_score[i] = skipped ? -INFINITY : sum;
+                }
             }
         }
         __syncthreads();

@@ -920,8 +920,10 @@ def run_ours(args):
             from seeded_inputs import PAGED_DECODE as PD, make_paged_cache
             dq, dk, dv, dtable, dlens = make_paged_cache(dw.B, dw.H, [dw.Nkv] * dw.B, dw.d,
                                                          PD["page_size"], dw_r.seed, device="cuda")
-            if ws > 1:   # the query row is the same on every rank; the cache is the rank's shard
-                dq = make_paged_cache(dw.B, dw.H, [dw.Nkv] * dw.B, dw.d, PD["page_size"],
+            if ws > 1:
+                # the query row is the same on every rank (the base seed's first draw, which
+                # does not depend on the cache size); the cache is the rank's shard
+                dq = make_paged_cache(dw.B, dw.H, [1] * dw.B, dw.d, PD["page_size"],
                                       dw.seed, device="cuda")[0]
         else:
             dq, dk, dv = make_workload(dw_r, device="cuda")

@@ -141,3 +141,10 @@ def test_query_draw_does_not_depend_on_the_key_count():
     q_small = make_qkv(2, 3, 1, 1, 16, seed=4)[0]
     q_full = make_qkv(2, 3, 1, 4097, 16, seed=4)[0]
     assert torch.equal(q_small, q_full)
+
+
+def test_paged_query_draw_does_not_depend_on_the_cache_size():
+    from seeded_inputs import make_paged_cache
+    q_small = make_paged_cache(2, 3, [1, 1], 16, 16, seed=5)[0]
+    q_full = make_paged_cache(2, 3, [300, 77], 16, 16, seed=5)[0]
+    assert torch.equal(q_small, q_full)

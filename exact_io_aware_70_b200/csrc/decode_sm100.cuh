@@ -103,9 +103,6 @@ __device__ __forceinline__ void axpy8(float p, const uint4& kv, float (&acc)[8])
 #ifndef EATTN_DECODE_MIN_CTAS
 #define EATTN_DECODE_MIN_CTAS 3
 #endif
-#ifndef EATTN_DECODE_PAGED_MIN_CTAS
-#define EATTN_DECODE_PAGED_MIN_CTAS 4
-#endif
 
 template <int D>
 struct DecodeTraits {
@@ -171,7 +168,7 @@ __device__ __forceinline__ int reduce_owner_index(int glane) {
 // The paged instantiation is held to 64 registers (4 CTAs per SM): measured
 // 6.63 TB/s against 4.83 TB/s at its unconstrained 80 registers (3 CTAs).
 template <int D, bool PAGED>
-__global__ void __launch_bounds__(256, PAGED ? EATTN_DECODE_PAGED_MIN_CTAS : EATTN_DECODE_MIN_CTAS)
+__global__ void __launch_bounds__(256, PAGED ? 4 : EATTN_DECODE_MIN_CTAS)
     attn_decode_partials_kernel(const DecodeParams p) {
     using T = DecodeTraits<D>;
     constexpr int LPR = T::kLanesPerRow, RPP = T::kRowsPerPass, NB = T::kBatch;

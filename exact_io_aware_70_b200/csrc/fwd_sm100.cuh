@@ -22,16 +22,20 @@
 //   * Warp 8 is the TMA producer (lane 0 issues): Q tiles once per unit,
 //     then K_j and V_j tiles into a ring of shared-memory slots, 128-byte
 //     swizzled, completion counted on mbarriers.
-//   * Warp 9 issues every tcgen05.mma from lane 0, with shared-memory
-//     descriptors precomputed per tile and advanced by constant offsets. A
-//     tcgen05.mma costs the issuing thread about 48 cycles (measured), close
-//     to the 64 cycles one 128x128x16 MMA keeps the tensor core busy, so this
-//     thread's loop is kept as short as possible: S_t = Q_t K_j^T into
-//     tensor memory (fp32, 128x128), and O_t += P_t V_j with P_t read straight
-//     from tensor memory (bf16, aliased over S_t's first 64 columns).
+//   * Lane 0 of warp 9 issues the tcgen05.mma products (head dim 128), or
+//     lane 0 of warp 9 those of Q tile 0 and lane 0 of warp 10 those of Q tile
+//     1 (head dim 64, fwd_mma_split), with shared-memory descriptors
+//     precomputed per tile and advanced by constant offsets: S_t = Q_t K_j^T
+//     into tensor memory (fp32, 128x128), and O_t += P_t V_j with P_t read
+//     straight from tensor memory (bf16). The issuing thread blocks while the
+//     tensor core's queue is full, so it spends about as long on a product as
+//     the tensor core does (64 cycles for 128x128x16, measured; a 128x64x16
+//     product still takes about 56), and every commit and wait on its path
+//     delays the next product.
 //   * 384 threads = 3 warpgroups; warps 10-11 only complete the third
-//     warpgroup so it can shrink its register budget (setmaxnreg) in favour
-//     of the two softmax warpgroups.
+//     warpgroup (warp 10 lane 0 issues tile 1's products at head dim 64) so
+//     it can shrink its register budget (setmaxnreg) in favour of the two
+//     softmax warpgroups.
 //   * Warps 0-3 and 4-7 are the softmax groups of Q tile 0 and Q tile 1, one
 //     thread per query row (= TMEM lane). While one group exponentiates its
 //     tile, the tensor core works on the other tile's products (ping-pong).
@@ -57,10 +61,11 @@
 //     measured slower). K_j and V_j complete on one barrier, and each Q tile is
 //     released to the producer right after its last S product of the unit.
 //   * Tensor memory columns, head dim 128: S0 [0,128), S1 [128,256), O0
-//     [256,384), O1 [384,512); S_t(j+1) overwrites P_t(j), so it is issued
-//     after P_t(j) V. Head dim 64: three score buffers [0,384) used in
-//     rotation, O0 [384,448), O1 [448,512); S_t(j+1) is computed one step
-//     ahead, while the softmax group still works on S_t(j) (fwd_mma_ahead).
+//     [256,384), O1 [384,512), P_t over S_t's first 64 columns; S_t(j+1)
+//     overwrites P_t(j), so it is issued after P_t(j) V. Head dim 64: tile t
+//     owns [256t, 256t+256): S_t, then P_t in its own 64 columns, then O_t;
+//     S_t(j+1) is computed as soon as the softmax group has read S_t(j) into
+//     registers, while it still exponentiates it (fwd_mma_split).
 //   * Epilogue: O / l in bf16 goes through a 2 KB shared-memory block per
 //     warp so that each global store instruction writes whole rows' 64-byte
 //     pieces (full 32-byte sectors) rather than one 16-byte piece of 32 rows.
@@ -122,8 +127,28 @@ struct FwdParams {
 #ifndef EATTN_SBUFS_AHEAD
 #define EATTN_SBUFS_AHEAD 1
 #endif
+// 1: (bf16) P is stored to TMEM once per tile (64 columns) after both halves'
+//    exponentials, instead of once per half
+#ifndef EATTN_P_STORE_ONCE
+#define EATTN_P_STORE_ONCE 0
+#endif
+// 1: at head dim 64 each Q tile has its own MMA-issuing thread and its own
+//    tensor-memory columns for S, P and O (fwd_mma_split), so the two tiles'
+//    chains of products no longer wait on each other; 0: one issuing thread
+//    for both tiles.
+#ifndef EATTN_SPLIT_ISSUE
+#define EATTN_SPLIT_ISSUE 1
+#endif
+// 1: (bf16 inputs) the softmax groups signal "P handed over", "S read" and
+//    "O free" with one barrier arrival per warp (after a warp-level sync)
+//    rather than one per thread; 0: every thread arrives. (For e4m3 inputs
+//    the per-warp form made the compiler spill and measured 5% slower.)
+#ifndef EATTN_WARP_ARRIVE
+#define EATTN_WARP_ARRIVE 1
+#endif
 // 1: two sets of Q tiles where shared memory allows (see FwdTraits::kQBufs).
-//    Measured slower on gpt2_1k (45.1 against 43.0 us), so off.
+//    With one issuing thread it measured slower on gpt2_1k (45.1 against
+//    43.0 us), so there it is off; the split issue always uses two sets.
 #ifndef EATTN_Q_DOUBLE
 #define EATTN_Q_DOUBLE 0
 #endif
@@ -176,6 +201,9 @@ struct FwdTraits {
     static_assert(2 * 128 * kSoftmaxRegs + 128 * kOtherRegs <= kThreads * kLaunchRegs,
                   "register split exceeds the launch allocation");
     static constexpr int kNumBars = 2 * kSlots + 27;   // FwdBars<kSlots>::kCount
+    // One MMA-issuing thread per Q tile (head dim 64: 2 x (128 S + 64 P + D O)
+    // columns fit in the 512).
+    static constexpr bool kSplit = EATTN_SPLIT_ISSUE && 2 * (128 + 64 + D) <= 512;
     // epilogue staging: one 32-row x 64-byte (32 bf16 columns) block per softmax warp
     static constexpr int kStageWarpBytes = 32 * 64;
     static constexpr int kStageBytes = EATTN_STAGE_O ? 8 * kStageWarpBytes : 0;
@@ -183,7 +211,7 @@ struct FwdTraits {
     // 64, and e4m3 inputs), so that the next unit's Q is loaded while this
     // unit still runs instead of after its last S product
     static constexpr int kQBufs =
-        (EATTN_Q_DOUBLE &&
+        ((EATTN_Q_DOUBLE || kSplit) &&
          1024 + (4 + kSlots) * kTileBytes + kStageBytes + kNumBars * 8 + 32 <= 232448) ? 4 : 2;
     static constexpr int kSmemBytes =
         1024 + (kQBufs + kSlots) * kTileBytes + kStageBytes + kNumBars * 8 + 16 + 16;
@@ -195,9 +223,20 @@ struct FwdTraits {
     // With three (head dim 64: 3 x 128 + 2 x 64 = 512) the S products rotate
     // over the buffers in issue order and S_t(j+1) is computed ahead, while
     // the softmax still works on S_t(j) (see fwd_mma).
-    static constexpr int kSBufs = (EATTN_SBUFS_AHEAD && 3 * 128 + 2 * D <= 512) ? 3 : 2;
-    static constexpr uint32_t kColS0 = 0, kColS1 = 128;
-    static constexpr uint32_t kColO0 = 128 * kSBufs, kColO1 = 128 * kSBufs + D;
+    // With one issuing thread per tile (kSplit) tile t has its own S buffer at
+    // column 256 t, P (bf16 pairs or e4m3 quads) at 256 t + 128 instead of
+    // over S, and O at 256 t + 192: S_t(j+1) may then be computed as soon as
+    // the softmax has read S_t(j), while it still works on it.
+    static constexpr int kSBufs = (!kSplit && EATTN_SBUFS_AHEAD && 3 * 128 + 2 * D <= 512) ? 3 : 2;
+    static constexpr uint32_t kColS0 = 0, kColS1 = kSplit ? 256 : 128;
+    static constexpr uint32_t kColP0 = kSplit ? 128 : kColS0, kColP1 = kSplit ? 384 : kColS1;
+    static constexpr uint32_t kColO0 = kSplit ? 192 : 128 * kSBufs;
+    static constexpr uint32_t kColO1 = kSplit ? 448 : 128 * kSBufs + D;
+    // readers of a unit-ring entry: the MMA issuer(s) and one lane of each softmax warp
+    static constexpr int kUnitReaders = kSplit ? 10 : 9;
+    // arrivals of one softmax warpgroup on p_lo/p_hi, o_free and (kSplit) "S free"
+    static constexpr bool kWarpArrive = EATTN_WARP_ARRIVE && !FP8;
+    static constexpr int kArrivals = kWarpArrive ? 4 : 128;
 };
 
 // One exponent pair in every kPolyEvery<D, FP8> goes to the FMA-pipe polynomial
@@ -326,7 +365,8 @@ struct FwdBars {
     __device__ __forceinline__ uint32_t unit_empty(int i) const { return base + 8 * (2 * S + 17 + i); }
     // three score buffers only: S_t products alternate between s_full(t) and
     // s_full_b(t) (one may complete before the softmax has seen the other);
-    // pv_done(t) completes with every P_t V product
+    // pv_done(t) completes with every P_t V product. With one issuer per tile
+    // s_full_b(t) is instead "S_t free": the softmax group has read S_t.
     __device__ __forceinline__ uint32_t s_full_b(int t) const { return base + 8 * (2 * S + 19 + t); }
     __device__ __forceinline__ uint32_t pv_done(int t) const { return base + 8 * (2 * S + 21 + t); }
     // barrier and parity of tile t's c-th score product (c counted over the CTA's life)
@@ -345,10 +385,6 @@ struct FwdBars {
     }
     uint8_t* unit_ring_ptr;
 };
-
-// Readers of a unit-ring entry: the MMA issuer and one lane of each of the 8
-// softmax warps.
-constexpr int kUnitReaders = 9;
 
 // Next unit for a consumer role. Dynamic deal: waits for ring entry k, reads
 // it and releases the entry (the MMA issuer and lane 0 of each softmax warp
@@ -637,6 +673,103 @@ done: {
 }
 }
 
+// One issuing thread per Q tile (FwdTraits::kSplit): this thread issues
+// every product of tile t. Per K/V step j of a unit the order is
+//   S_t(j) (once the softmax group has read S_t(j-1)), then P_t(j-1) V_{j-1},
+// so S_t(j) is computed while the group still exponentiates S_t(j-1), and
+// P_t(j-1) V waits only for this tile's own hand-over, never for the other
+// tile's. K and V slots are released by both issuers (kv_empty counts two
+// arrivals); a tile with fewer steps than the unit still waits for each K/V
+// pair, in order, and releases it at once.
+template <int D, bool CAUSAL, bool FP8>
+__device__ void fwd_mma_split(const FwdParams& p, uint32_t tbase, uint32_t sQ, uint32_t sKV,
+                              const FwdBars<FwdTraits<D, FP8>::kSlots>& b, uint32_t leader,
+                              volatile int* abort_flag, int t) {
+    using T = FwdTraits<D, FP8>;
+    static_assert(T::kSplit && !EATTN_SPLIT_P && EATTN_KV_PAIR_BARRIER, "split issue layout");
+    constexpr uint64_t kTileStep = T::kTileBytes >> 4;
+    const uint64_t dq0 = fwd_sdesc<T>(sQ, 16);
+    const uint64_t dk0 = fwd_sdesc<T>(sKV, 16);                       // K-major K tile
+    const uint64_t dv0 = fwd_sdesc<T>(sKV, T::kPanelBytes);           // MN-major V tile
+    const uint32_t tS = tbase + (t ? T::kColS1 : T::kColS0);
+    const uint32_t tP = tbase + (t ? T::kColP1 : T::kColP0);
+    const uint32_t tO = tbase + (t ? T::kColO1 : T::kColO0);
+    uint32_t kv_iter = 0;           // K and V tiles of all units so far (two per step)
+    uint32_t q_use[2] = {0, 0};     // units that used Q set 0 / set 1
+    uint32_t o_use = 0, s_cnt = 0, p_cnt = 0;
+    for (uint32_t k = 0;; ++k) {
+        int u;
+        if (!fwd_next_unit(p, b, k, true, abort_flag, &u)) goto done;
+        if (u < 0) break;
+        {
+            const FwdUnit x = fwd_unit<CAUSAL>(u, p);
+            const int n = x.n[t];
+            const int qi = 2 * (T::kQBufs == 4 ? (int)(k & 1) : 0) + t;
+            const uint32_t qset = qi >> 1;
+            if (!role_wait(b.q_full(qi), q_use[qset] & 1, abort_flag)) goto done;
+            ++q_use[qset];
+            if (n == 0) mma_commit_w(b.q_empty(qi), leader);
+            // P_t(i) V_i, V_i in ring slot vslot
+            auto issue_pv = [&](int i, uint32_t vslot) -> bool {
+                if (!role_wait(b.p_hi(t), p_cnt & 1, abort_flag)) return false;
+                ++p_cnt;
+                if (i == 0 && o_use > 0 && !role_wait(b.o_free(t), (o_use - 1) & 1, abort_flag))
+                    return false;
+                tc_fence_after_sync();
+                fwd_issue_pv<D, FP8>(tO, tP, dv0 + vslot * kTileStep, i > 0, 0, leader);
+                fwd_issue_pv<D, FP8>(tO, tP, dv0 + vslot * kTileStep, true, 1, leader);
+                mma_commit_w(b.pv_done(t), leader);
+                if (i == n - 1) mma_commit_w(b.o_final(t), leader);
+                mma_commit_w(b.kv_empty(vslot), leader);
+                return true;
+            };
+            uint32_t prev_vslot = 0;
+            for (int j = 0; j < x.nmax; ++j) {
+                const uint32_t kslot = kv_iter % T::kSlots;
+                const uint32_t vslot = (kv_iter + 1) % T::kSlots;
+                if (!role_wait(b.kv_full(kslot), (kv_iter / T::kSlots) & 1, abort_flag)) goto done;
+                kv_iter += 2;
+                if (j < n) {
+                    // S_t(j) overwrites S_t(j-1): wait until the softmax group has read it
+                    if (s_cnt > 0 && !role_wait(b.s_full_b(t), (s_cnt - 1) & 1, abort_flag))
+                        goto done;
+                    tc_fence_after_sync();
+                    fwd_issue_s<D, FP8>(tS, dq0 + qi * kTileStep, dk0 + kslot * kTileStep, leader);
+                    mma_commit_w(b.s_full(t), leader);
+                    ++s_cnt;
+                    if (j == n - 1) mma_commit_w(b.q_empty(qi), leader);
+                    mma_commit_w(b.kv_empty(kslot), leader);
+                } else if (leader) {
+                    mbar_arrive(b.kv_empty(kslot));   // this tile does not read K_j
+                }
+                if (j >= 1) {
+                    if (j - 1 < n) {
+                        if (!issue_pv(j - 1, prev_vslot)) goto done;
+                    } else if (leader) {
+                        mbar_arrive(b.kv_empty(prev_vslot));
+                    }
+                }
+                prev_vslot = vslot;
+            }
+            if (x.nmax > 0) {
+                if (x.nmax - 1 < n) {
+                    if (!issue_pv(x.nmax - 1, prev_vslot)) goto done;
+                } else if (leader) {
+                    mbar_arrive(b.kv_empty(prev_vslot));
+                }
+            }
+            if (n > 0) ++o_use;
+        }
+    }
+done: {
+    // Every MMA this thread issued must finish before tensor memory is released
+    // (the drain barrier counts one arrival per issuing thread).
+    volatile int no_abort = 0;
+    mma_commit_w(b.drain(), leader);
+    mbar_wait(b.drain(), 0, &no_abort, &g_attn_status);
+}
+}
+
 // Run by the whole MMA warp with converged control flow; lane 0 issues.
 template <int D, bool CAUSAL, bool FP8>
 __device__ void fwd_mma(const FwdParams& p, uint32_t tbase, uint32_t sQ, uint32_t sKV,
@@ -740,6 +873,22 @@ done: {
 }
 
 // --------------------------------------------------------------- softmax --
+// Arrival of a softmax warp on a barrier the MMA issuer waits for, after this
+// thread's tensor-memory accesses (made complete by the caller's tcgen05
+// wait) are ordered before it. Counts FwdTraits::kArrivals per warpgroup.
+template <bool kPerWarp>
+__device__ __forceinline__ void softmax_arrive(uint32_t bar, int lane) {
+    tc_fence_before_sync();
+    if (kPerWarp) {
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar);
+    } else {
+        mbar_arrive(bar);
+    }
+}
+
+
+
 // Epilogue store of one 32-column chunk of this warp's 32 rows. Lane l holds
 // row l's 32 bf16 values (w, 16 words). They go through the warp's 2 KB
 // staging block so that the global stores are row-contiguous: each store
@@ -814,6 +963,8 @@ __device__ void fwd_softmax(const FwdParams& p, uint32_t tbase,
                 tbase + lane_off +
                 (T::kSBufs == 3 ? ((s_base + fwd_s_pos(x, t, j)) % 3) * 128
                                 : (t ? T::kColS1 : T::kColS0));
+            // P_t(j): over S_t(j)'s first columns, or in its own columns (kSplit)
+            const uint32_t tP = T::kSplit ? tbase + lane_off + (t ? T::kColP1 : T::kColP0) : tS;
             if (!warp_wait(b.template s_bar<T::kSBufs>(t, s_cnt),
                            FwdBars<T::kSlots>::template s_parity<T::kSBufs>(s_cnt), abort_flag))
                 return;
@@ -822,6 +973,8 @@ __device__ void fwd_softmax(const FwdParams& p, uint32_t tbase,
             uint32_t sr[128];
             tmem_ld128(tS, sr);
             tmem_wait_ld128(sr);
+            if (T::kSplit)   // S_t(j) is in registers: its issuer may compute S_t(j+1) over it
+                softmax_arrive<T::kWarpArrive>(b.s_full_b(t), lane);
             {
                 // columns c >= lim of this tile are masked (-inf) for this row
                 const int lim = max(-1, min(128, kv_lim - j * 128));
@@ -849,6 +1002,8 @@ __device__ void fwd_softmax(const FwdParams& p, uint32_t tbase,
             const f32x2_t c2x2 = f2_pack(c2, c2);
             const f32x2_t nbx2 = f2_pack(-base, -base);
             f32x2_t lsum_a = f2_pack(0.f, 0.f), lsum_b = f2_pack(0.f, 0.f);
+            // bf16 with EATTN_P_STORE_ONCE: both halves' P words, stored together
+            [[maybe_unused]] uint32_t pk_all[(EATTN_P_STORE_ONCE && !FP8) ? 64 : 1];
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
                 uint32_t pk[FP8 ? 16 : 32];     // bf16 pairs or e4m3 quads
@@ -881,6 +1036,13 @@ __device__ void fwd_softmax(const FwdParams& p, uint32_t tbase,
                     else
                         lsum_a = f2_add(lsum_a, f2_pack(e0, e1));
                 }
+                // One issuer per tile: P_t(j) overwrites P_t(j-1), so P_t(j-1) V must be
+                // complete (it is issued as soon as P_t(j-1) is handed over, a whole
+                // softmax earlier, so this wait rarely waits); the rescale below
+                // needs the same product complete.
+                if (T::kSplit && h == 0 && j > 0 &&
+                    !warp_wait(b.pv_done(t), (p_cnt - 1) & 1, abort_flag))
+                    return;
                 if (h == 0 && any_need && j > 0) {
                     // Rescale O_t by alpha (1 for rows whose max did not move)
                     // before any of P_t(j) V is released. O_t must hold P_t(j-1) V:
@@ -888,7 +1050,7 @@ __device__ void fwd_softmax(const FwdParams& p, uint32_t tbase,
                     // covers it; with three, S_t(j) was issued before it, so wait
                     // for its own completion (P_t(j) is not released yet, so that
                     // barrier cannot be a phase further on).
-                    if (T::kSBufs == 3 &&
+                    if (T::kSBufs == 3 && !T::kSplit &&
                         !warp_wait(b.pv_done(t), (p_cnt - 1) & 1, abort_flag))
                         return;
                     tc_fence_after_sync();
@@ -903,16 +1065,21 @@ __device__ void fwd_softmax(const FwdParams& p, uint32_t tbase,
                         tmem_st32(tO + c, orr);
                     }
                 }
-                if constexpr (FP8)
-                    tmem_st16(tS + 16 * h, pk);
-                else
-                    tmem_st32(tS + 32 * h, pk);
+                if constexpr (FP8) {
+                    tmem_st16(tP + 16 * h, pk);
+                } else if constexpr (EATTN_P_STORE_ONCE) {
+#pragma unroll
+                    for (int q = 0; q < 32; ++q) pk_all[32 * h + q] = pk[q];
+                    if (h == 1) tmem_st64(tP, pk_all);
+                } else {
+                    tmem_st32(tP + 32 * h, pk);
+                }
                 if (EATTN_SPLIT_P || h == 1) {
                     tmem_wait_st();
-                    tc_fence_before_sync();
                     // three score buffers: P_t tiles alternate between p_hi and p_lo
-                    mbar_arrive(T::kSBufs == 3 ? ((p_cnt & 1) ? bar_plo : bar_phi)
-                                               : (h == 0 ? bar_plo : bar_phi));
+                    softmax_arrive<T::kWarpArrive>(T::kSBufs == 3 ? ((p_cnt & 1) ? bar_plo : bar_phi)
+                                                  : (h == 0 ? bar_plo : bar_phi),
+                                   lane);
                 }
             }
             ++p_cnt;
@@ -957,8 +1124,7 @@ __device__ void fwd_softmax(const FwdParams& p, uint32_t tbase,
                         dst[k4] = make_uint4(w[4 * k4], w[4 * k4 + 1], w[4 * k4 + 2], w[4 * k4 + 3]);
                 }
             }
-            tc_fence_before_sync();
-            mbar_arrive(bar_ofree);
+            softmax_arrive<T::kWarpArrive>(bar_ofree, lane);
             ++o_use;
         } else if (row_valid && dcheck(x.bh < p.BH)) {
             uint4* dst = reinterpret_cast<uint4*>(orow);
@@ -999,22 +1165,22 @@ __global__ void __launch_bounds__(384, 1)
     if (threadIdx.x == 0) {
         for (int i = 0; i < T::kSlots; ++i) {
             mbar_init(b.kv_full(i), 1);
-            mbar_init(b.kv_empty(i), 1);
+            mbar_init(b.kv_empty(i), T::kSplit ? 2 : 1);   // one arrival per issuing thread
         }
         for (int t = 0; t < 2; ++t) {
             mbar_init(b.q_full(t), 1);
             mbar_init(b.q_empty(t), 1);
             mbar_init(b.s_full(t), 1);
-            mbar_init(b.p_lo(t), 128);
-            mbar_init(b.p_hi(t), 128);
+            mbar_init(b.p_lo(t), T::kArrivals);
+            mbar_init(b.p_hi(t), T::kArrivals);
             mbar_init(b.o_final(t), 1);
-            mbar_init(b.o_free(t), 128);
+            mbar_init(b.o_free(t), T::kArrivals);
         }
-        mbar_init(b.drain(), 1);
+        mbar_init(b.drain(), T::kSplit ? 2 : 1);
         for (int i = 0; i < 2; ++i) {
             mbar_init(b.unit_full(i), 1);
-            mbar_init(b.unit_empty(i), kUnitReaders);
-            mbar_init(b.s_full_b(i), 1);
+            mbar_init(b.unit_empty(i), T::kUnitReaders);
+            mbar_init(b.s_full_b(i), T::kSplit ? T::kArrivals : 1);   // kSplit: "S_t free"
             mbar_init(b.pv_done(i), 1);
             mbar_init(b.q_full(2 + i), 1);
             mbar_init(b.q_empty(2 + i), 1);
@@ -1044,7 +1210,10 @@ __global__ void __launch_bounds__(384, 1)
         const bool issuer_thread = EATTN_WARP_ISSUE ? true : lane == 0;
         if (warp == 8 && issuer_thread)
             fwd_producer<D, CAUSAL, FP8>(p, &tm_q, &tm_k, &tm_v, sQ, sKV, b, lane == 0, abort_flag);
-        else if (warp == 9 && issuer_thread) {
+        else if constexpr (T::kSplit) {
+            if ((warp == 9 || warp == 10) && issuer_thread)   // warp 9: tile 0, warp 10: tile 1
+                fwd_mma_split<D, CAUSAL, FP8>(p, tbase, sQ, sKV, b, lane == 0, abort_flag, warp - 9);
+        } else if (warp == 9 && issuer_thread) {
             if constexpr (T::kSBufs == 3)
                 fwd_mma_ahead<D, CAUSAL, FP8>(p, tbase, sQ, sKV, b, lane == 0, abort_flag);
             else

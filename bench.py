@@ -14,7 +14,8 @@ the L2 size is written before every timed step, outside the kernels' CUDA
 events, and the line adds ``hot``, the same kernels back to back.
 
 ``--workload prefill_8k_bwd`` (or another ``*_bwd``) times the backward pass
-(dQ, dK, dV) of that prefill workload instead, one attn_bwd call per step.
+(dQ, dK, dV) of that prefill workload instead, one attn_bwd call per step
+(attn_bwd_deterministic with ``--deterministic``).
 
 ``--workload prefill_8k_fp8`` times the forward pass on e4m3 inputs
 (attn_fwd_fp8) of that workload.
@@ -694,10 +695,14 @@ def run_bwd(args):
               lse.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), w.B, w.H, w.Nq, w.Nkv,
               w.d, int(w.causal), w.scale, work.data_ptr(), work.numel(), sp)
 
+    det = bool(args.deterministic)
+    entry = L.attn_bwd_deterministic if det else L.attn_bwd
+    name = "attn_bwd_deterministic" if det else "attn_bwd"
+
     def step():
-        rc = L.attn_bwd(*args_c)
+        rc = entry(*args_c)
         if rc != 0:
-            raise RuntimeError(f"attn_bwd: {ea.attn_strerror(rc)}")
+            raise RuntimeError(f"{name}: {ea.attn_strerror(rc)}")
 
     flush = L2Flusher([q, k, v, o, do, lse, dq, dk, dv, work], dev, bool(args.batch))
     for _ in range(args.warmup):
@@ -719,7 +724,8 @@ def run_bwd(args):
         def e2e_step():
             for dst, src in zip((q, k, v, o, do, lse), hin):
                 dst.copy_(src, non_blocking=True)
-            ea.attn_bwd(q, k, v, o, do, lse, dq, dk, dv, w.causal, w.scale, work)
+            ea.attn_bwd(q, k, v, o, do, lse, dq, dk, dv, w.causal, w.scale, work,
+                        deterministic=det)
             for dst, src in zip(hout, (dq, dk, dv)):
                 dst.copy_(src, non_blocking=True)
 
@@ -737,7 +743,7 @@ def run_bwd(args):
             raise RuntimeError("device status reported an error in the e2e region")
         e2e = {"value": None, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
                "d2h_bytes_per_step": d2h, "ms_per_step": ems, "steps": E,
-               "path": "pinned host -> copy -> attn_bwd -> copy back, per step, CUDA events"}
+               "path": f"pinned host -> copy -> {name} -> copy back, per step, CUDA events"}
     vals = max_over_ranks([total_ms, call_ms] + ([e2e["ms_per_step"]] if e2e else []) +
                           ([hot_ms] if hot_ms is not None else []), device=dev)
     total_ms, call_ms = vals[0], vals[1]
@@ -753,10 +759,12 @@ def run_bwd(args):
         return 0
     pk = peaks()
     a = bwd_flops(w) / (call_ms * 1e-3) / 1e12
-    roof = {"kernel": "attn_bwd (preprocess + attn_bwd_sm100 + postprocess, timed as one call)",
+    roof = {"kernel": (f"{name} ({'kv bound + ' if det else ''}preprocess + attn_bwd_sm100 + "
+                       "postprocess, timed as one call)"),
             "bound": "tensor", "achieved": a, "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
             "frac": a / pk["bf16_tflops"], "frac_of_sustained": a / pk["bf16_tflops_sustained"],
-            "traffic": recorded_traffic().get(("attn_bwd_sm100", args.workload)),
+            "traffic": recorded_traffic().get(
+                ("attn_bwd_sm100", args.workload + ("_deterministic" if det else ""))),
             "algorithmic_bytes": bwd_bytes(w), "algorithmic_flops": bwd_flops(w), "ms": call_ms}
     line = {
         "metric": "attn bwd TFLOP/s & % BF16 tensor peak",
@@ -765,12 +773,13 @@ def run_bwd(args):
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": {"workload": args.workload, "B": w.B, "H": w.H, "N": w.Nq, "d": w.d,
                    "causal": w.causal, "flop_per_step": bwd_flops(w), "l2": flush.note,
+                   "entry": name,
                    "parallelism": (f"batch partitioned: one {w.B}-entry slice per GPU x{ws}"
                                    if ws > 1 else "1 GPU")},
         "roofline": roof,
         "peaks": dict(pk, note="of measured" if pk["source"] == "measured" else "of fallback"),
         "clocks": clk.summary(max_mhz_default=1965.0),
-        "gpu_launches": 3 * K, "e2e": e2e,
+        "gpu_launches": (4 if det else 3) * K, "e2e": e2e,
     }
     if hot_ms is not None:
         line["hot"] = {"value": ws * bwd_flops(w) / (hot_ms * 1e-3) / 1e12,
@@ -1245,6 +1254,8 @@ def main():
                     help="default line only: skip timing tiny, gpt2_1k and prefill_16k")
     ap.add_argument("--no-naive", action="store_true",
                     help="skip the naive materialising attention comparison")
+    ap.add_argument("--deterministic", action="store_true",
+                    help="*_bwd workloads: time attn_bwd_deterministic (fixed-point dQ)")
     ap.add_argument("--cpu-budget", type=float, default=8.0,
                     help="seconds of oracle work for the CPU baseline")
     args = ap.parse_args()

@@ -8,7 +8,7 @@ has not been built; there is no fallback implementation.
 Entry points (same names as the C ABI):
   attn_fwd(q, k, v, o, lse, causal, scale)            prefill forward, O and LSE
   attn_fwd_fp8(q, k, v, q_descale, k_descale, v_descale, o, lse, causal, scale)
-  attn_bwd(q, k, v, o, dout, lse, dq, dk, dv, causal, scale, workspace)
+  attn_bwd(q, k, v, o, dout, lse, dq, dk, dv, causal, scale, workspace[, deterministic])
   attn_bwd_workspace_bytes(B, H, Nq, d)
   attn_decode_partials(q, k, v, o_part, lse_part, scale, num_splits)
   attn_lse_merge(o_part, lse_part, o, lse)
@@ -72,6 +72,8 @@ lib.attn_bwd_workspace_bytes.restype = _sz
 lib.attn_bwd_workspace_bytes.argtypes = [_i, _i, _i, _i]
 lib.attn_bwd.restype = _i
 lib.attn_bwd.argtypes = [_vp] * 9 + [_i] * 6 + [_f, _vp, _sz, _vp]
+lib.attn_bwd_deterministic.restype = _i
+lib.attn_bwd_deterministic.argtypes = lib.attn_bwd.argtypes
 lib.attn_status.restype = _i
 lib.attn_status.argtypes = [_vp]
 
@@ -245,9 +247,10 @@ def attn_bwd_workspace_bytes(B: int, H: int, Nq: int, d: int) -> int:
 
 
 def attn_bwd(q, k, v, o, dout, lse, dq, dk, dv, causal: bool, scale: float, workspace,
-             stream=None) -> None:
+             stream=None, deterministic: bool = False) -> None:
     """dQ, dK, dV of sum(dO*O). q/o/dout/dq [B,H,Nq,d], k/v/dk/dv [B,H,Nkv,d] bf16; lse [B,H,Nq] fp32;
-    workspace: a device buffer of at least attn_bwd_workspace_bytes(B, H, Nq, d) bytes."""
+    workspace: a device buffer of at least attn_bwd_workspace_bytes(B, H, Nq, d) bytes.
+    deterministic: call attn_bwd_deterministic (dQ bit-identical from run to run)."""
     import torch
     B, H, Nq, d = q.shape
     Nkv = k.shape[2]
@@ -257,13 +260,15 @@ def attn_bwd(q, k, v, o, dout, lse, dq, dk, dv, causal: bool, scale: float, work
         raise ValueError("attn_bwd: inconsistent shapes")
     if not workspace.is_contiguous():
         raise ValueError("attn_bwd: workspace must be contiguous")
-    _check(lib.attn_bwd(_tensor(q, torch.bfloat16, "q"), _tensor(k, torch.bfloat16, "k"),
-                        _tensor(v, torch.bfloat16, "v"), _tensor(o, torch.bfloat16, "o"),
-                        _tensor(dout, torch.bfloat16, "dout"), _tensor(lse, torch.float32, "lse"),
-                        _tensor(dq, torch.bfloat16, "dq"), _tensor(dk, torch.bfloat16, "dk"),
-                        _tensor(dv, torch.bfloat16, "dv"), B, H, Nq, Nkv, d, int(bool(causal)),
-                        float(scale), ctypes.c_void_p(workspace.data_ptr()),
-                        workspace.numel() * workspace.element_size(), _stream(stream)), "attn_bwd")
+    fn = lib.attn_bwd_deterministic if deterministic else lib.attn_bwd
+    _check(fn(_tensor(q, torch.bfloat16, "q"), _tensor(k, torch.bfloat16, "k"),
+              _tensor(v, torch.bfloat16, "v"), _tensor(o, torch.bfloat16, "o"),
+              _tensor(dout, torch.bfloat16, "dout"), _tensor(lse, torch.float32, "lse"),
+              _tensor(dq, torch.bfloat16, "dq"), _tensor(dk, torch.bfloat16, "dk"),
+              _tensor(dv, torch.bfloat16, "dv"), B, H, Nq, Nkv, d, int(bool(causal)),
+              float(scale), ctypes.c_void_p(workspace.data_ptr()),
+              workspace.numel() * workspace.element_size(), _stream(stream)),
+           "attn_bwd_deterministic" if deterministic else "attn_bwd")
 
 
 def attn_status(stream=None) -> int:

@@ -209,6 +209,13 @@ attn_status_t launch_bwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUt
     }
     const long long prows = (long long)p.BH * p.NqPad;
     constexpr int kRowsPerBlock = 256 / (D / 8);
+    if (p.deterministic) {
+        if (cudaMemsetAsync(p.bound, 0, 3 * sizeof(unsigned), stream) != cudaSuccess)
+            return ATTN_ERR_CUDA;
+        const long long kvrows = (long long)p.BH * p.Nkv;
+        attn_bwd_kv_bound_kernel<D>
+            <<<(unsigned)((kvrows + kRowsPerBlock - 1) / kRowsPerBlock), 256, 0, stream>>>(p);
+    }
     attn_bwd_preprocess_kernel<D>
         <<<(unsigned)((prows + kRowsPerBlock - 1) / kRowsPerBlock), 256, 0, stream>>>(p);
     const long long rows = (long long)p.BH * p.Nq;
@@ -524,13 +531,16 @@ attn_status_t attn_decode_splitkv(const void* q, const void* k, const void* v, v
 size_t attn_bwd_workspace_bytes(int B, int H, int Nq, int d) {
     if (B < 1 || H < 1 || Nq < 1 || (d != 64 && d != 128)) return 0;
     const size_t prow = (size_t)B * H * (((size_t)Nq + 63) / 64 * 64);
-    return 2 * ((prow * 4 + 255) / 256 * 256) + (size_t)B * H * Nq * d * 4;
+    return 2 * ((prow * 4 + 255) / 256 * 256) + 256 + (size_t)B * H * Nq * d * 8;
 }
 
-attn_status_t attn_bwd(const void* q, const void* k, const void* v, const void* o,
-                       const void* dout, const float* lse, void* dq, void* dk, void* dv, int B,
-                       int H, int Nq, int Nkv, int d, int causal, float scale, void* workspace,
-                       size_t workspace_bytes, void* stream) {
+}  // extern "C"
+
+namespace {
+attn_status_t bwd_entry(const void* q, const void* k, const void* v, const void* o,
+                        const void* dout, const float* lse, void* dq, void* dk, void* dv, int B,
+                        int H, int Nq, int Nkv, int d, int causal, float scale, void* workspace,
+                        size_t workspace_bytes, void* stream, bool deterministic) {
     if (!q || !k || !v || !o || !dout || !lse || !dq || !dk || !dv || !workspace)
         return ATTN_ERR_INVALID_ARG;
     if (causal != 0 && causal != 1) return ATTN_ERR_INVALID_ARG;
@@ -558,7 +568,11 @@ attn_status_t attn_bwd(const void* q, const void* k, const void* v, const void* 
     p.lse = lse;
     p.delta = static_cast<float*>(workspace);
     p.lse2 = reinterpret_cast<float*>(static_cast<char*>(workspace) + pbytes);
-    p.dq_acc = reinterpret_cast<float*>(static_cast<char*>(workspace) + 2 * pbytes);
+    p.bound = reinterpret_cast<unsigned*>(static_cast<char*>(workspace) + 2 * pbytes);
+    p.dq_acc = static_cast<char*>(workspace) + 2 * pbytes + 256;
+    p.deterministic = deterministic ? 1 : 0;
+    p.k = static_cast<const uint16_t*>(k);
+    p.v = static_cast<const uint16_t*>(v);
     p.NqPad = NqPad;
     p.dq = static_cast<uint16_t*>(dq);
     p.dk = static_cast<uint16_t*>(dk);
@@ -574,6 +588,26 @@ attn_status_t attn_bwd(const void* q, const void* k, const void* v, const void* 
                       : launch_bwd<128, false>(tq, tk, tv, tdo, p, st);
     return causal ? launch_bwd<64, true>(tq, tk, tv, tdo, p, st)
                   : launch_bwd<64, false>(tq, tk, tv, tdo, p, st);
+}
+}  // namespace
+
+extern "C" {
+
+attn_status_t attn_bwd(const void* q, const void* k, const void* v, const void* o,
+                       const void* dout, const float* lse, void* dq, void* dk, void* dv, int B,
+                       int H, int Nq, int Nkv, int d, int causal, float scale, void* workspace,
+                       size_t workspace_bytes, void* stream) {
+    return bwd_entry(q, k, v, o, dout, lse, dq, dk, dv, B, H, Nq, Nkv, d, causal, scale,
+                     workspace, workspace_bytes, stream, false);
+}
+
+attn_status_t attn_bwd_deterministic(const void* q, const void* k, const void* v, const void* o,
+                                     const void* dout, const float* lse, void* dq, void* dk,
+                                     void* dv, int B, int H, int Nq, int Nkv, int d, int causal,
+                                     float scale, void* workspace, size_t workspace_bytes,
+                                     void* stream) {
+    return bwd_entry(q, k, v, o, dout, lse, dq, dk, dv, B, H, Nq, Nkv, d, causal, scale,
+                     workspace, workspace_bytes, stream, true);
 }
 
 attn_status_t attn_selftest_wait_timeout(unsigned limit_us, void* stream) {

@@ -10,10 +10,13 @@
 //   dV = P^T dO;  dP = dO V^T;  D_i = sum_c dO_ic O_ic;  dS = P o (dP - D);
 //   dQ = scale * dS K;  dK = scale * dS^T Q.
 //
-// Three kernels:
+// Three kernels, four in the deterministic form:
+//   0. (deterministic form) attn_bwd_kv_bound: the largest |K| element and the
+//      largest V row norm, for the dQ accumulator's fixed-point scale (below);
 //   1. attn_bwd_preprocess: D = rowsum(dO o O) and LSE * log2(e) into padded
 //      per-head rows (so a 64-row block of either is one aligned 256-byte
-//      copy), and zeroing of the fp32 dQ accumulator;
+//      copy), zeroing of the dQ accumulator and (deterministic form) the
+//      largest dO row norm;
 //   2. attn_bwd_sm100: one CTA per (batch*head, 128-key block j), looping over
 //      the 64-row query blocks that can see block j, computed transposed:
 //      S^T = K_j Q_i^T and dP^T = V_j dO_i^T (M = the 128 keys, N = 64
@@ -21,10 +24,23 @@
 //      can stay in tensor memory as the A operand of dV += P^T dO_i and
 //      dK += dS^T Q_i. dS^T also goes to shared memory as the B operand of
 //      dQ_i^T = K_j^T dS^T (M = head dim), whose rows two reduction warpgroups
-//      add into the fp32 dQ accumulator, 128 contiguous bytes per
-//      instruction. Two tensor-memory stages let the tensor core work on one
-//      query block while the P/dS warps work on the next.
+//      add into the dQ accumulator. Two tensor-memory stages let the tensor
+//      core work on one query block while the P/dS warps work on the next.
 //   3. attn_bwd_postprocess: dQ = bf16(scale * accumulator).
+// The dQ accumulator is fp32, added to with fp32 atomics, so the last bits of
+// dQ depend on the order in which the CTAs add. The deterministic form
+// (attn_bwd_deterministic) makes it fixed point instead: int64 multiples of
+// 2^-F, added with integer atomics; integer addition is exact and
+// associative, so dQ is the same bits whatever the order. F is set per launch
+// from a bound on every partial sum of dQ_ic / scale, from the inputs alone:
+//   |sum_j dS_ij K_jc| <= max|K| * sum_j P_ij |dP_ij - D_i|
+//                      <= max|K| * (max_j |dO_i . V_j| + |dO_i . O_i|)
+//                      <= 2 max|K| max_i ||dO_i|| max_j ||V_j||
+// (Cauchy-Schwarz, sum_j P_ij <= 1, and O_i a convex combination of the V_j);
+// with a factor 2 for the bf16 rounding of P, dS and O, the bound B gives
+// F = 61 - ceil(log2 2B), so every partial sum times 2^F stays below 2^61
+// and the rounding of a contribution to the grid (2^-F / 2 <= B 2^-62) is far
+// below bf16's resolution of dQ.
 // Every mbarrier wait is bounded, as in the forward kernel.
 #pragma once
 
@@ -41,7 +57,11 @@ struct BwdParams {
     const float* lse;      // fp32 [BH, Nq]      (preprocess)
     float* delta;          // fp32 [BH, NqPad]: D_i, 0 past Nq
     float* lse2;           // fp32 [BH, NqPad]: LSE_i * log2(e); +inf past Nq or with no key
-    float* dq_acc;         // fp32 [BH, Nq, D]
+    void* dq_acc;          // [BH, Nq, D]: fp32, or int64 multiples of 2^-F (deterministic)
+    int deterministic;     // 1: the fixed-point dQ accumulator
+    unsigned* bound;       // [3]: max|K|, max ||dO_i||, max ||V_j|| (fp32 bits; zeroed first)
+    const uint16_t* k;     // bf16 [BH, Nkv, D]  (kv_bound)
+    const uint16_t* v;     // bf16 [BH, Nkv, D]  (kv_bound)
     uint16_t* dq;          // bf16 [BH, Nq, D]
     uint16_t* dk;          // bf16 [BH, Nkv, D]
     uint16_t* dv;          // bf16 [BH, Nkv, D]
@@ -50,6 +70,52 @@ struct BwdParams {
     float scale;           // softmax scale
     float scale_log2;      // scale * log2(e)
 };
+
+// ------------------------------------------------------------- dQ bound --
+// Largest of v over the warp, folded into *dst (v >= 0, so the fp32 bits of
+// non-negative values order like the values).
+__device__ __forceinline__ void bwd_max_into(unsigned* dst, float v) {
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, off));
+    if ((threadIdx.x & 31) == 0) atomicMax(dst, __float_as_uint(v));
+}
+
+// 2^F of the dQ accumulator (see the file header), from the three maxima.
+__device__ __forceinline__ int bwd_dq_exponent(const unsigned* bound) {
+    const float b = 2.f * __uint_as_float(bound[0]) * __uint_as_float(bound[1]) *
+                    __uint_as_float(bound[2]);
+    int e = 0;
+    frexpf(2.f * b, &e);   // 2B < 2^e (e = 0 for B = 0)
+    return min(120, max(-60, 61 - e));
+}
+
+__device__ __forceinline__ float bwd_bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bwd_bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
+
+// One thread per 8 elements of a K and a V row; D/8 threads per row; rows of
+// [BH, Nkv].
+template <int D>
+__global__ void __launch_bounds__(256) attn_bwd_kv_bound_kernel(const BwdParams p) {
+    constexpr int LPR = D / 8;
+    const long long row = (long long)blockIdx.x * (256 / LPR) + threadIdx.x / LPR;
+    const int cc = threadIdx.x % LPR;
+    float kmax = 0.f, vsq = 0.f;
+    if (row < (long long)p.BH * p.Nkv) {
+        const uint4 a = *reinterpret_cast<const uint4*>(p.k + row * D + cc * 8);
+        const uint4 g = *reinterpret_cast<const uint4*>(p.v + row * D + cc * 8);
+        const uint32_t av[4] = {a.x, a.y, a.z, a.w}, gv[4] = {g.x, g.y, g.z, g.w};
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            kmax = fmaxf(kmax, fmaxf(fabsf(bwd_bf16_lo(av[k])), fabsf(bwd_bf16_hi(av[k]))));
+            vsq = fmaf(bwd_bf16_lo(gv[k]), bwd_bf16_lo(gv[k]), vsq);
+            vsq = fmaf(bwd_bf16_hi(gv[k]), bwd_bf16_hi(gv[k]), vsq);
+        }
+    }
+#pragma unroll
+    for (int off = LPR / 2; off > 0; off >>= 1) vsq += __shfl_xor_sync(0xffffffffu, vsq, off);
+    bwd_max_into(&p.bound[0], kmax);
+    bwd_max_into(&p.bound[2], sqrtf(vsq));
+}
 
 // ------------------------------------------------------------ preprocess --
 // One thread per 8 elements of a row; D/8 threads per row; rows of [BH, NqPad].
@@ -64,23 +130,29 @@ __global__ void __launch_bounds__(256) attn_bwd_preprocess_kernel(const BwdParam
     const int i = in_range ? (int)(row % p.NqPad) : 0;
     const bool real = in_range && i < p.Nq && dcheck(bh < p.BH);
     const long long grow = bh * p.Nq + i;
-    float acc = 0.f;
+    float acc = 0.f, gsq = 0.f;
     if (real) {
         const uint4 a = *reinterpret_cast<const uint4*>(p.o + grow * D + cc * 8);
         const uint4 g = *reinterpret_cast<const uint4*>(p.dout + grow * D + cc * 8);
         const uint32_t av[4] = {a.x, a.y, a.z, a.w}, gv[4] = {g.x, g.y, g.z, g.w};
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
-            acc = fmaf(__uint_as_float(av[k] << 16), __uint_as_float(gv[k] << 16), acc);
-            acc = fmaf(__uint_as_float(av[k] & 0xFFFF0000u), __uint_as_float(gv[k] & 0xFFFF0000u),
-                       acc);
+            acc = fmaf(bwd_bf16_lo(av[k]), bwd_bf16_lo(gv[k]), acc);
+            acc = fmaf(bwd_bf16_hi(av[k]), bwd_bf16_hi(gv[k]), acc);
+            gsq = fmaf(bwd_bf16_lo(gv[k]), bwd_bf16_lo(gv[k]), gsq);
+            gsq = fmaf(bwd_bf16_hi(gv[k]), bwd_bf16_hi(gv[k]), gsq);
         }
-        float4* z = reinterpret_cast<float4*>(p.dq_acc + grow * D + cc * 8);
-        z[0] = make_float4(0.f, 0.f, 0.f, 0.f);
-        z[1] = make_float4(0.f, 0.f, 0.f, 0.f);
+        // 8 elements of 4 or 8 bytes
+        uint4* z = reinterpret_cast<uint4*>(static_cast<char*>(p.dq_acc) +
+                                            (grow * D + cc * 8) * (p.deterministic ? 8 : 4));
+        for (int k = 0; k < (p.deterministic ? 4 : 2); ++k) z[k] = make_uint4(0, 0, 0, 0);
     }
 #pragma unroll
-    for (int off = LPR / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+    for (int off = LPR / 2; off > 0; off >>= 1) {
+        acc += __shfl_xor_sync(0xffffffffu, acc, off);
+        gsq += __shfl_xor_sync(0xffffffffu, gsq, off);
+    }
+    if (p.deterministic) bwd_max_into(&p.bound[1], sqrtf(gsq));
     if (in_range && cc == 0) {
         p.delta[row] = real ? acc : 0.f;
         // a row with no visible key (LSE = -inf) or past Nq gets P = 2^(s - inf) = 0
@@ -94,12 +166,29 @@ template <int D>
 __global__ void __launch_bounds__(256) attn_bwd_postprocess_kernel(const BwdParams p) {
     const long long i = ((long long)blockIdx.x * 256 + threadIdx.x) * 8;
     if (i >= (long long)p.BH * p.Nq * D) return;
-    const float4 a = *reinterpret_cast<const float4*>(p.dq_acc + i);
-    const float4 b = *reinterpret_cast<const float4*>(p.dq_acc + i + 4);
-    const float s = p.scale;
+    float f[8];
+    if (p.deterministic) {
+        // scale * 2^-F: a power of two times scale, exact in fp32 for F in [-60, 120]
+        const float s = p.scale * ldexpf(1.f, -bwd_dq_exponent(p.bound));
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            const longlong2 a = reinterpret_cast<const longlong2*>(p.dq_acc)[i / 2 + k];
+            f[2 * k] = __ll2float_rn(a.x) * s;
+            f[2 * k + 1] = __ll2float_rn(a.y) * s;
+        }
+    } else {
+#pragma unroll
+        for (int k = 0; k < 2; ++k) {
+            const float4 a = reinterpret_cast<const float4*>(p.dq_acc)[i / 4 + k];
+            f[4 * k] = a.x * p.scale;
+            f[4 * k + 1] = a.y * p.scale;
+            f[4 * k + 2] = a.z * p.scale;
+            f[4 * k + 3] = a.w * p.scale;
+        }
+    }
     *reinterpret_cast<uint4*>(p.dq + i) =
-        make_uint4(pack_bf16x2(a.x * s, a.y * s), pack_bf16x2(a.z * s, a.w * s),
-                   pack_bf16x2(b.x * s, b.y * s), pack_bf16x2(b.z * s, b.w * s));
+        make_uint4(pack_bf16x2(f[0], f[1]), pack_bf16x2(f[2], f[3]), pack_bf16x2(f[4], f[5]),
+                   pack_bf16x2(f[6], f[7]));
 }
 
 // ------------------------------------------------------------ main kernel --
@@ -166,6 +255,12 @@ __device__ __forceinline__ int bwd_first_qblock(int j, const BwdParams& p) {
 
 __device__ __forceinline__ void red_add_f32(float* addr, float v) {
     asm volatile("red.global.add.f32 [%0], %1;" ::"l"(addr), "f"(v) : "memory");
+}
+// Adds v, rounded to the accumulator's grid (v * 2^F to the nearest integer),
+// to a fixed-point dQ element.
+__device__ __forceinline__ void red_add_fixed(long long* addr, float v, float two_f) {
+    const long long x = __float2ll_rn(v * two_f);
+    asm volatile("red.global.add.u64 [%0], %1;" ::"l"(addr), "l"(x) : "memory");
 }
 
 __device__ __forceinline__ void fence_proxy_async_smem() {
@@ -360,7 +455,10 @@ __global__ void __launch_bounds__(640, 1)
         const int cols = 32 * ((warp - 8) >> 2);   // this warp's first query column
         const int c = quarter * 32 + lane;
         const uint32_t lane_off = uint32_t(quarter * 32) << 16;
-        float* dq_head = p.dq_acc + (size_t)bh * p.Nq * D + (c < D ? c : 0);
+        const size_t head_off = (size_t)bh * p.Nq * D + (c < D ? c : 0);
+        float* dq_head = static_cast<float*>(p.dq_acc) + head_off;
+        long long* dq_head64 = static_cast<long long*>(p.dq_acc) + head_off;
+        const float two_f = p.deterministic ? ldexpf(1.f, bwd_dq_exponent(p.bound)) : 0.f;
         for (int s = 0; s < nsteps; ++s) {
             const int x = s & 1;
             bool ok = mbar_wait(b.dq_full(x), (s >> 1) & 1, abort_flag, &g_attn_status);
@@ -374,14 +472,26 @@ __global__ void __launch_bounds__(640, 1)
             const int row0 = (i0 + s) * T::kQRows + cols;
             if (quarter * 32 < D) {
                 float* dq_rows = dq_head + (size_t)row0 * D;
+                long long* dq_rows64 = dq_head64 + (size_t)row0 * D;
                 const int nr = p.Nq - row0;   // rows of this block inside the head
                 if (nr >= 32 && dcheck(row0 + 32 <= p.Nq && bh < p.BH)) {
+                    if (p.deterministic) {
 #pragma unroll
-                    for (int e = 0; e < 32; ++e) red_add_f32(dq_rows + e * D, __uint_as_float(v[e]));
+                        for (int e = 0; e < 32; ++e)
+                            red_add_fixed(dq_rows64 + e * D, __uint_as_float(v[e]), two_f);
+                    } else {
+#pragma unroll
+                        for (int e = 0; e < 32; ++e) red_add_f32(dq_rows + e * D, __uint_as_float(v[e]));
+                    }
                 } else if (nr < 32) {
 #pragma unroll
                     for (int e = 0; e < 32; ++e)
-                        if (e < nr) red_add_f32(dq_rows + e * D, __uint_as_float(v[e]));
+                        if (e < nr) {
+                            if (p.deterministic)
+                                red_add_fixed(dq_rows64 + e * D, __uint_as_float(v[e]), two_f);
+                            else
+                                red_add_f32(dq_rows + e * D, __uint_as_float(v[e]));
+                        }
                 }
             }
         }

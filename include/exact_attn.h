@@ -269,8 +269,11 @@ attn_status_t attn_decode_splitkv_noalloc(const void *q, const void *k, const vo
  * Backward pass: bytes of device workspace attn_bwd needs, or 0 if the
  * arguments are invalid. Layout (owned by the caller, 256-byte aligned), with
  * NqPad = Nq rounded up to a multiple of 64: fp32 D [B, H, NqPad] and fp32
- * LSE * log2(e) [B, H, NqPad], each padded to 256 bytes, then the fp32 dQ
- * accumulator [B, H, Nq, d]. Nothing in it needs initialising.
+ * LSE * log2(e) [B, H, NqPad], each padded to 256 bytes, 256 bytes for the
+ * three maxima that set attn_bwd_deterministic's accumulator scale, then the
+ * dQ accumulator: fp32 [B, H, Nq, d] for attn_bwd, int64 fixed point for
+ * attn_bwd_deterministic (the size covers the int64 form). Nothing in it
+ * needs initialising.
  */
 size_t attn_bwd_workspace_bytes(int B, int H, int Nq, int d);
 
@@ -300,12 +303,30 @@ size_t attn_bwd_workspace_bytes(int B, int H, int Nq, int d);
  *   Three kernels run on `stream` in order: D, LSE * log2(e) and zeroing of
  *   the accumulator; the main kernel (one CTA per 128-key block and head,
  *   64-row query blocks); and the dQ conversion. dQ is summed with fp32 atomic
- *   adds, so its last bits may vary from run to run; dK and dV do not.
+ *   adds, so its last bits may vary from run to run; dK and dV do not
+ *   (attn_bwd_deterministic gives bit-identical dQ too).
  */
 attn_status_t attn_bwd(const void *q, const void *k, const void *v, const void *o,
                        const void *dout, const float *lse, void *dq, void *dk, void *dv, int B,
                        int H, int Nq, int Nkv, int d, int causal, float scale, void *workspace,
                        size_t workspace_bytes, void *stream);
+
+/*
+ * attn_bwd whose dQ, like dK and dV, is the same bits on every run: same
+ * arguments, workspace and errors. dQ is summed in a fixed-point int64
+ * accumulator (multiples of 2^-F) with integer atomic adds, which are exact in
+ * any order; F is chosen per call so that no partial sum can overflow, from
+ * the bound |sum_j dS_ij K_jc| <= 2 max|K| max_i ||dO_i|| max_j ||V_j|| (times
+ * 2 for bf16 rounding), computed by an extra kernel over K and V and by the
+ * first kernel over dO (a 12-byte memset of the workspace comes first).
+ * Inputs must be finite. The integer atomics cost more than fp32 ones (about
+ * 1.5x the backward's time at 8K).
+ */
+attn_status_t attn_bwd_deterministic(const void *q, const void *k, const void *v, const void *o,
+                                     const void *dout, const float *lse, void *dq, void *dk,
+                                     void *dv, int B, int H, int Nq, int Nkv, int d, int causal,
+                                     float scale, void *workspace, size_t workspace_bytes,
+                                     void *stream);
 
 /*
  * Synchronises `stream`, then returns and clears the device status word:

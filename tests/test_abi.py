@@ -132,16 +132,22 @@ def test_bwd_rejects_bad_arguments_without_launching(ea):
     L = ea.lib
     p = 0x10000
     ws_need = ea.attn_bwd_workspace_bytes(1, 2, 300, 128)
-    assert ws_need == 2 * ((2 * 320 * 4 + 255) // 256 * 256) + 2 * 300 * 128 * 4
+    # D and LSE * log2(e) rows padded to 64 and to 256 bytes, 256 bytes of maxima,
+    # then the dQ accumulator in its int64 form
+    assert ws_need == 2 * ((2 * 320 * 4 + 255) // 256 * 256) + 256 + 2 * 300 * 128 * 8
     assert ea.attn_bwd_workspace_bytes(1, 2, 300, 96) == 0
     assert ea.attn_bwd_workspace_bytes(1, 2, 0, 128) == 0
+    for fn in (L.attn_bwd, L.attn_bwd_deterministic):
+        _bwd_bad_arguments(ea, fn, p, ws_need)
 
+
+def _bwd_bad_arguments(ea, fn, p, ws_need):
     def call(ws_bytes=ws_need, **kw):
         a = dict(dict(q=p, k=p, v=p, o=p, do=p, lse=p, dq=p, dk=p, dv=p, ws=p, B=1, H=2, Nq=300,
                       Nkv=300, d=128, causal=1, scale=0.088), **kw)
-        return L.attn_bwd(a["q"], a["k"], a["v"], a["o"], a["do"], a["lse"], a["dq"], a["dk"],
-                          a["dv"], a["B"], a["H"], a["Nq"], a["Nkv"], a["d"], a["causal"],
-                          a["scale"], a["ws"], ws_bytes, None)
+        return fn(a["q"], a["k"], a["v"], a["o"], a["do"], a["lse"], a["dq"], a["dk"],
+                  a["dv"], a["B"], a["H"], a["Nq"], a["Nkv"], a["d"], a["causal"],
+                  a["scale"], a["ws"], ws_bytes, None)
 
     assert call(do=None) == ea.ATTN_ERR_INVALID_ARG
     assert call(ws=None) == ea.ATTN_ERR_INVALID_ARG

@@ -11,7 +11,7 @@ from tests.parity import compare_grad, grad_error_bound
 pytestmark = pytest.mark.gpu
 
 
-def run_bwd(q, k, v, do, causal, scale, guard=256):
+def run_bwd(q, k, v, do, causal, scale, guard=256, deterministic=False):
     """Forward then backward through the C ABI; outputs surrounded by canary bands."""
     m = gpu_util.ea()
     B, H, Nq, d = q.shape
@@ -27,7 +27,7 @@ def run_bwd(q, k, v, do, causal, scale, guard=256):
     dk = outs[1].view(B, H, Nkv, d)
     dv = outs[2].view(B, H, Nkv, d)
     ws = torch.empty(m.attn_bwd_workspace_bytes(B, H, Nq, d), dtype=torch.uint8, device="cuda")
-    m.attn_bwd(q, k, v, o, do, lse, dq, dk, dv, causal, scale, ws)
+    m.attn_bwd(q, k, v, o, do, lse, dq, dk, dv, causal, scale, ws, deterministic=deterministic)
     assert m.attn_status() == 0
     for buf, n in bufs:
         assert torch.all(buf[:guard] == -77.0) and torch.all(buf[guard + n:] == -77.0), \
@@ -103,13 +103,65 @@ def test_bwd_prefill_8k_one_head():
 
 
 def test_bwd_dk_dv_deterministic():
-    """dK and dV have a fixed summation order; dQ goes through fp32 atomics."""
+    """dK and dV have a fixed summation order; attn_bwd's dQ goes through fp32 atomics."""
     scale = float(np.float32(1.0 / np.sqrt(128)))
     q, k, v = (t.cuda() for t in make_qkv(1, 4, 700, 700, 128, 11))
     do = make_dout(1, 4, 700, 128, 11, device="cuda")
     a = run_bwd(q, k, v, do, True, scale)
     b = run_bwd(q, k, v, do, True, scale)
     assert torch.equal(a[1], b[1]) and torch.equal(a[2], b[2])
+
+
+@pytest.mark.parametrize("d,causal", [(128, True), (64, False)])
+def test_bwd_deterministic_form(d, causal):
+    """attn_bwd_deterministic sums dQ in fixed point with integer atomics: every
+    gradient is the same bits on every run although 256 CTAs add into dQ in
+    whatever order they get there, and all three meet the error model (dK and
+    dV equal attn_bwd's bit for bit)."""
+    scale = float(np.float32(1.0 / np.sqrt(d)))
+    B, H, N = 2, 8, 2048
+    q, k, v = (t.cuda() for t in make_qkv(B, H, N, N, d, 11 + d))
+    do = make_dout(B, H, N, d, 11 + d, device="cuda")
+    runs = [run_bwd(q, k, v, do, causal, scale, deterministic=True) for _ in range(3)]
+    for r in runs[1:]:
+        for g in range(3):
+            assert torch.equal(runs[0][g], r[g]), ("dQ", "dK", "dV")[g]
+    dq, dk, dv, o = runs[0]
+    check_heads(q, k, v, do, o, dq, dk, dv, causal, scale, [(0, 0), (1, 7)],
+                f"deterministic d{d}")
+    fast = run_bwd(q, k, v, do, causal, scale)
+    assert torch.equal(fast[1], dk) and torch.equal(fast[2], dv)
+
+
+def test_bwd_deterministic_large_and_zero_gradients():
+    """The fixed-point scale follows the inputs: large gradients (V x 8, dO x 300, so
+    dQ about 2400 times its usual size; Q and K as usual, so the softmax is not
+    pushed to denormal probabilities) still meet the error model without
+    overflow, and dO = 0 gives exact zeros."""
+    B, H, N, d = 1, 2, 400, 64
+    scale = float(np.float32(1.0 / np.sqrt(d)))
+    q, k, v = (t.cuda() for t in make_qkv(B, H, N, N, d, 23))
+    v = (v.float() * 8).to(torch.bfloat16)
+    do = (make_dout(B, H, N, d, 23, device="cuda").float() * 300).to(torch.bfloat16)
+    dq, dk, dv, o = run_bwd(q, k, v, do, True, scale, deterministic=True)
+    check_heads(q, k, v, do, o, dq, dk, dv, True, scale, [(0, 0), (0, 1)], "large values")
+    dq0, dk0, dv0, _ = run_bwd(q, k, v, torch.zeros_like(do), True, scale, deterministic=True)
+    assert not torch.any(dq0) and not torch.any(dk0) and not torch.any(dv0)
+
+
+@pytest.mark.parametrize("B,H,Nq,Nkv,d,causal", [
+    (1, 2, 300, 300, 128, True),      # ragged tails
+    (1, 1, 520, 200, 128, True),      # leading rows see no key
+    (1, 1, 1, 1, 64, False),          # single element
+])
+def test_bwd_deterministic_edges(B, H, Nq, Nkv, d, causal):
+    scale = float(np.float32(1.0 / np.sqrt(d)))
+    seed = Nq * 3 + Nkv + d
+    q, k, v = (t.cuda() for t in make_qkv(B, H, Nq, Nkv, d, seed))
+    do = make_dout(B, H, Nq, d, seed, device="cuda")
+    dq, dk, dv, o = run_bwd(q, k, v, do, causal, scale, deterministic=True)
+    check_heads(q, k, v, do, o, dq, dk, dv, causal, scale,
+                [(b, h) for b in range(B) for h in range(H)], f"deterministic {Nq}x{Nkv}")
 
 
 def test_bwd_rejects_small_workspace():

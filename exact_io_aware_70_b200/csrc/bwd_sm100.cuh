@@ -80,14 +80,16 @@ __device__ __forceinline__ void bwd_max_into(unsigned* dst, float v) {
     if ((threadIdx.x & 31) == 0) atomicMax(dst, __float_as_uint(v));
 }
 
-// 2^F of the dQ accumulator (see the file header), from the three maxima.
+// F of the dQ accumulator's grid 2^-F (see the file header), from the three
+// maxima: with 2B = m 2^e, m in [1, 2) (e the unbiased exponent), 2B < 2^(e+1).
 __device__ __forceinline__ int bwd_dq_exponent(const unsigned* bound) {
     const float b = 2.f * __uint_as_float(bound[0]) * __uint_as_float(bound[1]) *
                     __uint_as_float(bound[2]);
-    int e = 0;
-    frexpf(2.f * b, &e);   // 2B < 2^e (e = 0 for B = 0)
-    return min(120, max(-60, 61 - e));
+    const int e = (int)((__float_as_uint(2.f * b) >> 23) & 0xFFu) - 127;
+    return min(120, max(-60, 60 - e));
 }
+// 2^f as an fp32 bit pattern, f in [-126, 127]
+__device__ __forceinline__ float bwd_pow2(int f) { return __uint_as_float((uint32_t)(f + 127) << 23); }
 
 __device__ __forceinline__ float bwd_bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bwd_bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
@@ -169,7 +171,7 @@ __global__ void __launch_bounds__(256) attn_bwd_postprocess_kernel(const BwdPara
     float f[8];
     if (p.deterministic) {
         // scale * 2^-F: a power of two times scale, exact in fp32 for F in [-60, 120]
-        const float s = p.scale * ldexpf(1.f, -bwd_dq_exponent(p.bound));
+        const float s = p.scale * bwd_pow2(-bwd_dq_exponent(p.bound));
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
             const longlong2 a = reinterpret_cast<const longlong2*>(p.dq_acc)[i / 2 + k];
@@ -458,7 +460,7 @@ __global__ void __launch_bounds__(640, 1)
         const size_t head_off = (size_t)bh * p.Nq * D + (c < D ? c : 0);
         float* dq_head = static_cast<float*>(p.dq_acc) + head_off;
         long long* dq_head64 = static_cast<long long*>(p.dq_acc) + head_off;
-        const float two_f = p.deterministic ? ldexpf(1.f, bwd_dq_exponent(p.bound)) : 0.f;
+        const float two_f = p.deterministic ? bwd_pow2(bwd_dq_exponent(p.bound)) : 0.f;
         for (int s = 0; s < nsteps; ++s) {
             const int x = s & 1;
             bool ok = mbar_wait(b.dq_full(x), (s >> 1) & 1, abort_flag, &g_attn_status);

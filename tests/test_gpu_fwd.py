@@ -34,6 +34,9 @@ SWEEP = [
     # per group, the last group short; then one head per group)
     (2, 4, 300, 21845, 128, True),
     (1, 3, 512, 65536, 128, False),
+    # head dim 64 (one issuing thread per Q tile) with long K/V rows: with the
+    # dynamic deal, groups of 5 heads of 5.6 MB of K/V, the last group short
+    (2, 4, 300, 21845, 64, True),
 ]
 
 
@@ -81,7 +84,7 @@ def schedule(monkeypatch, request):
 
 
 @pytest.mark.parametrize("schedule", ["dynamic", "static"], indirect=True)
-@pytest.mark.parametrize("shape", [SWEEP[i] for i in (1, 6, 9, 16, 18, 19, 20, 21)],
+@pytest.mark.parametrize("shape", [SWEEP[i] for i in (1, 6, 9, 16, 18, 19, 20, 21, 22)],
                          ids=lambda s: "B{}H{}q{}kv{}d{}c{}".format(*s[:5], int(s[5])))
 def test_fwd_sweep_both_schedules(shape, schedule):
     B, H, Nq, Nkv, d, causal = shape

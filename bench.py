@@ -587,29 +587,25 @@ def run_fp8(args):
         hout = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in (o, lse)]
         h2d = sum(t.numel() * t.element_size() for t in hin)
         d2h = sum(t.numel() * t.element_size() for t in hout)
-        q8, k8, v8, qd, kd, vd = ins
+        sets = [list(ins) + [o, lse], [torch.empty_like(t) for t in list(ins) + [o, lse]]]
 
-        def e2e_step():
-            for dst, src in zip(ins, hin):
-                dst.copy_(src, non_blocking=True)
-            ea.attn_fwd_fp8(q8, k8, v8, qd, kd, vd, o, lse, w.causal, w.scale)
-            for dst, src in zip(hout, (o, lse)):
-                dst.copy_(src, non_blocking=True)
+        def run(b):
+            q8, k8, v8, qd, kd, vd, O, Ls = sets[b]
+            ea.attn_fwd_fp8(q8, k8, v8, qd, kd, vd, O, Ls, w.causal, w.scale)
 
-        e2e_step()
-        torch.cuda.synchronize()
-        E = max(2, min(K, 3))
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        for _ in range(E):
-            e2e_step()
-        e1.record(stream)
-        torch.cuda.synchronize()
+        h2d_l = [(h, (sets[0][i], sets[1][i])) for i, h in enumerate(hin)]
+        d2h_l = [((sets[0][6 + i], sets[1][6 + i]), h) for i, h in enumerate(hout)]
+        pipelined_e2e(h2d_l, run, d2h_l, 2, stream)   # warm-up
+        E = max(4, min(K, 6))
+        ems = pipelined_e2e(h2d_l, run, d2h_l, E, stream)
+        del sets
         if ea.attn_status() != 0:
             raise RuntimeError("device status reported an error in the e2e region")
         e2e = {"value": None, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
-               "d2h_bytes_per_step": d2h, "ms_per_step": e0.elapsed_time(e1) / E, "steps": E,
-               "path": "pinned host -> copy -> attn_fwd_fp8 -> copy back, per step, CUDA events"}
+               "d2h_bytes_per_step": d2h, "ms_per_step": ems, "steps": E,
+               "path": "pinned host -> copy (own stream) -> attn_fwd_fp8 -> copy back (own "
+                       "stream), every step; two device buffer sets, so one step's copies "
+                       "overlap the neighbouring steps' kernels; CUDA events"}
     vals = max_over_ranks([total_ms, call_ms] + ([e2e["ms_per_step"]] if e2e else []) +
                           ([hot_ms] if hot_ms is not None else []), device=dev)
     total_ms, call_ms = vals[0], vals[1]
@@ -721,29 +717,27 @@ def run_bwd(args):
         h2d = sum(t.numel() * t.element_size() for t in hin)
         d2h = sum(t.numel() * t.element_size() for t in hout)
 
-        def e2e_step():
-            for dst, src in zip((q, k, v, o, do, lse), hin):
-                dst.copy_(src, non_blocking=True)
-            ea.attn_bwd(q, k, v, o, do, lse, dq, dk, dv, w.causal, w.scale, work,
-                        deterministic=det)
-            for dst, src in zip(hout, (dq, dk, dv)):
-                dst.copy_(src, non_blocking=True)
+        tset = [q, k, v, o, do, lse, dq, dk, dv]
+        sets = [tset, [torch.empty_like(t) for t in tset]]
 
-        e2e_step()
-        torch.cuda.synchronize()
-        E = max(2, min(K, 3))
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        for _ in range(E):
-            e2e_step()
-        e1.record(stream)
-        torch.cuda.synchronize()
-        ems = e0.elapsed_time(e1) / E
+        def run(b):
+            Q, Kt, V, O, DO, Ls, DQ, DK, DV = sets[b]
+            ea.attn_bwd(Q, Kt, V, O, DO, Ls, DQ, DK, DV, w.causal, w.scale, work,
+                        deterministic=det)
+
+        h2d_l = [(h, (sets[0][i], sets[1][i])) for i, h in enumerate(hin)]
+        d2h_l = [((sets[0][6 + i], sets[1][6 + i]), h) for i, h in enumerate(hout)]
+        pipelined_e2e(h2d_l, run, d2h_l, 2, stream)   # warm-up
+        E = max(4, min(K, 6))
+        ems = pipelined_e2e(h2d_l, run, d2h_l, E, stream)
+        del sets
         if ea.attn_status() != 0:
             raise RuntimeError("device status reported an error in the e2e region")
         e2e = {"value": None, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
                "d2h_bytes_per_step": d2h, "ms_per_step": ems, "steps": E,
-               "path": f"pinned host -> copy -> {name} -> copy back, per step, CUDA events"}
+               "path": f"pinned host -> copy (own stream) -> {name} -> copy back (own stream), "
+                       "every step; two device buffer sets, so one step's copies overlap the "
+                       "neighbouring steps' kernels; CUDA events"}
     vals = max_over_ranks([total_ms, call_ms] + ([e2e["ms_per_step"]] if e2e else []) +
                           ([hot_ms] if hot_ms is not None else []), device=dev)
     total_ms, call_ms = vals[0], vals[1]
@@ -796,6 +790,44 @@ def run_bwd(args):
 
 
 # ------------------------------------------------------------ GPU arm --
+def pipelined_e2e(h2d, run, d2h, E, stream):
+    """E end-to-end steps, each copying its inputs from pinned host memory to one
+    of two device buffer sets (h2d: [(host, (dev_a, dev_b)), ...]), running
+    run(b) on `stream` for buffer set b, and copying its outputs back (d2h:
+    [((dev_a, dev_b), host), ...]). The copies in and the copies out each have
+    their own stream, so step i+1's inputs travel while step i computes and
+    step i-1's outputs come back; events keep a buffer set from being refilled
+    before its outputs are out. Returns the ms per step (CUDA events, the
+    first copy in to the last copy out, divided by E)."""
+    import torch
+    s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream()
+    e_in = [torch.cuda.Event() for _ in range(2)]
+    e_run = [torch.cuda.Event() for _ in range(2)]
+    e_free = [torch.cuda.Event() for _ in range(2)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    t0.record(s_in)
+    for i in range(E):
+        b = i & 1
+        with torch.cuda.stream(s_in):
+            if i >= 2:
+                s_in.wait_event(e_free[b])
+            for host, devs in h2d:
+                devs[b].copy_(host, non_blocking=True)
+            e_in[b].record(s_in)
+        stream.wait_event(e_in[b])
+        run(b)
+        e_run[b].record(stream)
+        with torch.cuda.stream(s_out):
+            s_out.wait_event(e_run[b])
+            for devs, host in d2h:
+                host.copy_(devs[b], non_blocking=True)
+            e_free[b].record(s_out)
+    t1.record(s_out)
+    torch.cuda.synchronize()
+    return t0.elapsed_time(t1) / E
+
+
 def _maybe_batch(w, batch):
     import dataclasses
     return dataclasses.replace(w, B=batch) if batch else w
@@ -1058,55 +1090,57 @@ def run_ours(args):
             h2d += sum(t.numel() * t.element_size() for t in (hdq, hdk, hdv))
             d2h += sum(t.numel() * t.element_size() for t in (hdo, hdl))
 
-        def e2e_prefill():
-            q.copy_(hq, non_blocking=True)
-            k.copy_(hk, non_blocking=True)
-            v.copy_(hv, non_blocking=True)
-            ea.attn_fwd(q, k, v, o, lse, pw.causal, pw.scale)
-            ho.copy_(o, non_blocking=True)
-            hl.copy_(lse, non_blocking=True)
+        # a second device buffer set, so that one step's copies overlap another's kernels
+        E = max(4, min(K, 6))
+        acc = []
+        if pw:
+            q2, k2, v2, o2 = (torch.empty_like(t) for t in (q, k, v, o))
+            lse2 = torch.empty_like(lse)
+            pset = [(q, k, v, o, lse), (q2, k2, v2, o2, lse2)]
 
-        def e2e_decode():
-            dq.copy_(hdq, non_blocking=True)
-            dk.copy_(hdk, non_blocking=True)
-            dv.copy_(hdv, non_blocking=True)
-            if ws > 1:
-                # this rank's shard through the public API, then the exchange and the merge
-                if paged:
-                    ea.attn_decode_paged_partials(dq, dk, dv, dtable, dlens, po, pl, dw.scale, S)
+            def run_prefill(b):
+                Q, Kt, V, O, Ls = pset[b]
+                ea.attn_fwd(Q, Kt, V, O, Ls, pw.causal, pw.scale)
+
+            pipelined_e2e([(hq, (q, q2)), (hk, (k, k2)), (hv, (v, v2))], run_prefill,
+                          [((o, o2), ho), ((lse, lse2), hl)], 2, stream)   # warm-up
+            acc.append(pipelined_e2e([(hq, (q, q2)), (hk, (k, k2)), (hv, (v, v2))], run_prefill,
+                                     [((o, o2), ho), ((lse, lse2), hl)], E, stream))
+            del q2, k2, v2, o2, lse2, pset
+        if dw:
+            dq2, dk2, dv2, do2 = (torch.empty_like(t) for t in (dq, dk, dv, do))
+            dlse2 = torch.empty_like(dlse)
+            dset = [(dq, dk, dv, do, dlse), (dq2, dk2, dv2, do2, dlse2)]
+
+            def run_decode(b):
+                Q, Kt, V, O, Ls = dset[b]
+                if ws > 1:
+                    # this rank's shard through the public API, then the exchange and the merge
+                    if paged:
+                        ea.attn_decode_paged_partials(Q, Kt, V, dtable, dlens, po, pl, dw.scale, S)
+                    else:
+                        ea.attn_decode_partials(Q, Kt, V, po, pl, dw.scale, S)
+                    launch_gather()
+                    ea.attn_lse_merge_gathered(og, lg, O, Ls)
+                elif paged:
+                    ea.attn_decode_paged(Q, Kt, V, dtable, dlens, O, Ls, dw.scale, S, work)
                 else:
-                    ea.attn_decode_partials(dq, dk, dv, po, pl, dw.scale, S)
-                launch_gather()
-                ea.attn_lse_merge_gathered(og, lg, do, dlse)
-            elif paged:
-                ea.attn_decode_paged(dq, dk, dv, dtable, dlens, do, dlse, dw.scale, S, work)
-            else:
-                ea.attn_decode_splitkv(dq, dk, dv, do, dlse, dw.scale, S, work)
-            hdo.copy_(do, non_blocking=True)
-            hdl.copy_(dlse, non_blocking=True)
+                    ea.attn_decode_splitkv(Q, Kt, V, O, Ls, dw.scale, S, work)
 
-        parts = ([e2e_prefill] if pw else []) + ([e2e_decode] if dw else [])
-        for fn in parts:
-            fn()
-        torch.cuda.synchronize()
-        E = max(2, min(K, 3))
-        ep = [torch.cuda.Event(enable_timing=True) for _ in range(len(parts) + 1)]
-        acc = [0.0] * len(parts)
-        for _ in range(E):
-            for i, fn in enumerate(parts):
-                ep[i].record(stream)
-                fn()
-            ep[len(parts)].record(stream)
-            torch.cuda.synchronize()
-            for i in range(len(parts)):
-                acc[i] += ep[i].elapsed_time(ep[i + 1]) / E
+            dh2d = [(hdq, (dq, dq2)), (hdk, (dk, dk2)), (hdv, (dv, dv2))]
+            dd2h = [((do, do2), hdo), ((dlse, dlse2), hdl)]
+            pipelined_e2e(dh2d, run_decode, dd2h, 2, stream)   # warm-up
+            acc.append(pipelined_e2e(dh2d, run_decode, dd2h, E, stream))
+            del dq2, dk2, dv2, do2, dlse2, dset
         acc = max_over_ranks(acc, device=dev)
         if ea.attn_status() != 0:
             raise RuntimeError("device status reported an error in the e2e region")
         e2e = {"h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": sum(acc),
                "steps": E,
-               "path": "pinned host -> copy -> attn_fwd / attn_decode_splitkv -> copy back, "
-                       "per step, CUDA events on the launching stream"}
+               "path": "pinned host -> copy (own stream) -> attn_fwd / attn_decode_splitkv "
+                       "(launching stream) -> copy back (own stream), every step; two device "
+                       "buffer sets, so one step's copies overlap the neighbouring steps' "
+                       "kernels; CUDA events from the first copy in to the last copy out"}
         if pw:
             e2e["value"] = ws * prefill_flops(pw) / (acc[0] * 1e-3) / 1e12
             e2e["unit"] = "TFLOP/s"

@@ -264,11 +264,12 @@ class ClockSampler:
 # PTX helpers it includes). A recorded figure is used only while these files
 # hash to the value stored beside it.
 KERNEL_SOURCES = {
-    "attn_fwd_sm100": ("fwd_sm100.cuh", "ptx_sm100.cuh", "tmem_wide.cuh"),
+    # attn_api.cu: the host sets the unit deal and head groups, which move the traffic
+    "attn_fwd_sm100": ("fwd_sm100.cuh", "ptx_sm100.cuh", "tmem_wide.cuh", "attn_api.cu"),
     "attn_decode_partials": ("decode_sm100.cuh", "ptx_sm100.cuh"),
     "attn_lse_merge": ("decode_sm100.cuh", "ptx_sm100.cuh"),
     "attn_bwd_sm100": ("bwd_sm100.cuh", "ptx_sm100.cuh", "tmem_wide.cuh"),
-    "attn_fwd_sm100_e4m3": ("fwd_sm100.cuh", "ptx_sm100.cuh", "tmem_wide.cuh"),
+    "attn_fwd_sm100_e4m3": ("fwd_sm100.cuh", "ptx_sm100.cuh", "tmem_wide.cuh", "attn_api.cu"),
 }
 
 

@@ -127,9 +127,11 @@ int current_device() {
 std::atomic<unsigned> g_fwd_queue_rr{0};
 
 // Heads per group of the forward's unit order: as many heads as keep their
-// K and V within kFwdGroupBytes, so the CTAs in flight find them in L2.
+// K and V within EATTN_FWD_GROUP_BYTES, so the CTAs in flight find them in
+// L2. Measured at 16K (8 MB of K/V per head): 16, 32, 48, 64, 96 and 128 MB
+// groups ran 3.63, 3.55-3.59, 3.58, 3.50-3.54, 3.67 and 3.58 ms.
 #ifndef EATTN_FWD_GROUP_BYTES
-#define EATTN_FWD_GROUP_BYTES (32ll << 20)
+#define EATTN_FWD_GROUP_BYTES (64ll << 20)
 #endif
 int fwd_group_heads(int BH, int Nkv, int d, int elem_bytes) {
     const long long per_head = 2ll * Nkv * d * elem_bytes;

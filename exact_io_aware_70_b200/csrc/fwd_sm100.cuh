@@ -912,12 +912,15 @@ __device__ __forceinline__ void fwd_store_chunk(uint32_t stage, const uint32_t (
         st_shared_v4(stage + stage_slot(lane, k), w[4 * k], w[4 * k + 1], w[4 * k + 2],
                      w[4 * k + 3]);
     __syncwarp();
-#pragma unroll 1
+    // all four pieces read from the staging block first, then the four stores
+    uint4 val[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) val[i] = ld_shared_v4(stage + stage_slot(i * 8 + (lane >> 2), lane & 3));
+#pragma unroll
     for (int i = 0; i < 4; ++i) {
         const int r = i * 8 + (lane >> 2), k = lane & 3;
-        const uint4 val = ld_shared_v4(stage + stage_slot(r, k));
         uint16_t* dst = o_rows + (size_t)r * D + c + 8 * k;
-        if (r < valid_rows && dcheck(dst + 8 <= o_end)) *reinterpret_cast<uint4*>(dst) = val;
+        if (r < valid_rows && dcheck(dst + 8 <= o_end)) *reinterpret_cast<uint4*>(dst) = val[i];
     }
 }
 

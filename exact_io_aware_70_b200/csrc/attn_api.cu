@@ -153,7 +153,7 @@ int fwd_group_heads(int BH, int Nkv, int d, int elem_bytes) {
 
 template <int D, bool CAUSAL, bool FP8 = false>
 attn_status_t launch_fwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                         FwdParams p, cudaStream_t stream) {
+                         const CUtensorMap& to, FwdParams p, cudaStream_t stream) {
     using T = FwdTraits<D, FP8>;
     const int dev = current_device();
     if (dev < 0 || dev >= 64) return ATTN_ERR_CUDA;
@@ -187,7 +187,7 @@ attn_status_t launch_fwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUt
                         ? fwd_group_heads(p.BH, p.Nkv, D, T::kElemBytes)
                         : p.BH;
     p.queue_slot = (int)(g_fwd_queue_rr.fetch_add(1, std::memory_order_relaxed) % kFwdQueueSlots);
-    kern<<<grid, T::kThreads, T::kSmemBytes, stream>>>(tq, tk, tv, p);
+    kern<<<grid, T::kThreads, T::kSmemBytes, stream>>>(tq, tk, tv, to, p);
     return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
 
@@ -274,9 +274,10 @@ attn_status_t attn_fwd(const void* q, const void* k, const void* v, void* o, flo
         return ATTN_ERR_ALIGNMENT;
 
     const int BH = B * H;
-    CUtensorMap tq, tk, tv;
+    CUtensorMap tq, tk, tv, to;
+    // O: stored by the softmax warps as boxes of 32 rows x 64 columns
     if (!encode_bf16_map(&tq, q, BH, Nq, d) || !encode_bf16_map(&tk, k, BH, Nkv, d) ||
-        !encode_bf16_map(&tv, v, BH, Nkv, d))
+        !encode_bf16_map(&tv, v, BH, Nkv, d) || !encode_bf16_map(&to, o, BH, Nq, d, 32))
         return ATTN_ERR_CUDA;
     FwdParams p;
     p.o = static_cast<uint16_t*>(o);
@@ -292,10 +293,10 @@ attn_status_t attn_fwd(const void* q, const void* k, const void* v, void* o, flo
     p.scale_log2 = scale * kLog2e;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     if (d == 128)
-        return causal ? launch_fwd<128, true>(tq, tk, tv, p, st)
-                      : launch_fwd<128, false>(tq, tk, tv, p, st);
-    return causal ? launch_fwd<64, true>(tq, tk, tv, p, st)
-                  : launch_fwd<64, false>(tq, tk, tv, p, st);
+        return causal ? launch_fwd<128, true>(tq, tk, tv, to, p, st)
+                      : launch_fwd<128, false>(tq, tk, tv, to, p, st);
+    return causal ? launch_fwd<64, true>(tq, tk, tv, to, p, st)
+                  : launch_fwd<64, false>(tq, tk, tv, to, p, st);
 }
 
 attn_status_t attn_fwd_fp8(const void* q, const void* k, const void* v, const float* q_descale,
@@ -314,9 +315,9 @@ attn_status_t attn_fwd_fp8(const void* q, const void* k, const void* v, const fl
         !aligned(v_descale, 4))
         return ATTN_ERR_ALIGNMENT;
     const int BH = B * H;
-    CUtensorMap tq, tk, tv;
+    CUtensorMap tq, tk, tv, to;
     if (!encode_u8_map(&tq, q, BH, Nq, d) || !encode_u8_map(&tk, k, BH, Nkv, d) ||
-        !encode_u8_map(&tv, v, BH, Nkv, d))
+        !encode_u8_map(&tv, v, BH, Nkv, d) || !encode_bf16_map(&to, o, BH, Nq, d, 32))
         return ATTN_ERR_CUDA;
     FwdParams p;
     p.o = static_cast<uint16_t*>(o);
@@ -334,10 +335,10 @@ attn_status_t attn_fwd_fp8(const void* q, const void* k, const void* v, const fl
     p.scale_log2 = scale * kLog2e;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     if (d == 128)
-        return causal ? launch_fwd<128, true, true>(tq, tk, tv, p, st)
-                      : launch_fwd<128, false, true>(tq, tk, tv, p, st);
-    return causal ? launch_fwd<64, true, true>(tq, tk, tv, p, st)
-                  : launch_fwd<64, false, true>(tq, tk, tv, p, st);
+        return causal ? launch_fwd<128, true, true>(tq, tk, tv, to, p, st)
+                      : launch_fwd<128, false, true>(tq, tk, tv, to, p, st);
+    return causal ? launch_fwd<64, true, true>(tq, tk, tv, to, p, st)
+                  : launch_fwd<64, false, true>(tq, tk, tv, to, p, st);
 }
 
 attn_status_t attn_decode_partials(const void* q, const void* k, const void* v, float* o_part,

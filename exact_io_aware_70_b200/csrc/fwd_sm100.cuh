@@ -41,7 +41,9 @@
 //     tile, the tensor core works on the other tile's products (ping-pong).
 //     Each group also rescales its O tile in tensor memory when its running max
 //     grows by more than 2^8 (lazy rescaling: exact, since every p and l uses
-//     the same stale reference max), and runs the epilogue (O / l -> bf16,
+//     the same stale reference max), and runs the epilogue (O / l -> bf16
+//     through a per-warp shared-memory staging block: row-contiguous warp
+//     stores at head dim 128, one TMA tile store per warp at head dim 64;
 //     LSE = ln 2 * (m + log2 l)).
 //   * Exponentials are base 2 with log2(e) folded into the scale, computed
 //     with MUFU ex2 on pairs prepared by sm_100's packed f32x2 FMA; the row

@@ -903,14 +903,6 @@ __device__ __forceinline__ void softmax_arrive(uint32_t bar, int lane) {
 
 
 
-// Epilogue store of one 32-column chunk of this warp's 32 rows. Lane l holds
-// row l's 32 bf16 values (w, 16 words). They go through the warp's 2 KB
-// staging block so that the global stores are row-contiguous: each store
-// instruction writes 8 rows x 64 bytes (4 lanes per row, 16 bytes each), i.e.
-// whole 32-byte sectors, instead of 32 rows x 16 bytes. In the staging block,
-// rows 2p and 2p+1 share a 128-byte line and row r's 16-byte piece k sits in
-// slot (r & 1) * 4 + (k ^ (p & 3)) of its line, so that neither the row-wise
-// writes nor the piece-wise reads have bank conflicts.
 // TMA tile store shared -> global of one 3-D box ({x, y, z} element
 // coordinates, x a multiple of 64 bf16, never negative), tracked by this
 // thread's bulk async-group; rows past the map's extent are not written.
@@ -936,6 +928,15 @@ __device__ __forceinline__ void fence_async_shared() {
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
+
+// Epilogue store of one 32-column chunk of this warp's 32 rows. Lane l holds
+// row l's 32 bf16 values (w, 16 words). They go through the warp's 2 KB
+// staging block so that the global stores are row-contiguous: each store
+// instruction writes 8 rows x 64 bytes (4 lanes per row, 16 bytes each), i.e.
+// whole 32-byte sectors, instead of 32 rows x 16 bytes. In the staging block,
+// rows 2p and 2p+1 share a 128-byte line and row r's 16-byte piece k sits in
+// slot (r & 1) * 4 + (k ^ (p & 3)) of its line, so that neither the row-wise
+// writes nor the piece-wise reads have bank conflicts.
 __device__ __forceinline__ uint32_t stage_slot(int r, int k) {
     const int pr = r >> 1;
     return (uint32_t)((pr * 8 + (r & 1) * 4 + (k ^ (pr & 3))) * 16);

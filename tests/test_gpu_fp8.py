@@ -96,6 +96,7 @@ def _parity(B, H, Nq, Nkv, causal, seed, d=128):
     (1, 2, 1000, 777, False),
     (1, 1, 1, 1, False),
     (1, 3, 2048, 2048, True),     # many K/V tiles per row: lazy rescaling and ring wrap
+    (4, 40, 300, 300, True),      # 320 units: two or three per CTA, every second one ragged
 ])
 def test_fp8_matches_oracle(B, H, Nq, Nkv, causal, d):
     _parity(B, H, Nq, Nkv, causal, seed=Nq * 5 + Nkv + int(causal) + d, d=d)
